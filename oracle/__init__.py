@@ -1,0 +1,6 @@
+"""CPU oracle for multi-scale retention (test infrastructure only; see
+retention_oracle.py).  Only tests/, __graft_entry__.smoke() and bench.py's
+CPU legs may import it."""
+from .retention_oracle import (  # noqa: F401
+    chunkwise, decay_mask, group_norm, parallel, recurrent, rel_frobenius, step,
+)

@@ -1,0 +1,308 @@
+"""Pins of the CPU oracle to facts fixed outside the oracle itself.
+
+Each test checks the oracle against something it cannot agree with by
+construction: hand-worked values, brute force, textbook special cases,
+closed forms and the invariants the pages state (the three forms give the
+same output; state passes exactly across chunk boundaries).  The mutation
+tests at the end plant plausible mistakes in copies of the oracle's steps
+and show that a pin catches each of them.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from linear_recurrent_sequence_scale_b200 import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_worked.json")
+
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def _seq(a, d=None):
+    """[N] or [N,d] list -> [1,1,N,d] float64."""
+    x = np.asarray(a, dtype=np.float64)
+    if x.ndim == 1:
+        x = x[:, None]
+    return x[None, None]
+
+
+def _rand(rng, B, H, N, dk, dv, state=True):
+    q = rng.standard_normal((B, H, N, dk))
+    k = rng.standard_normal((B, H, N, dk))
+    v = rng.standard_normal((B, H, N, dv))
+    s = rng.standard_normal((B, H, dk, dv)) if state else None
+    return q, k, v, s
+
+
+# --- hand-worked values ------------------------------------------------------
+
+@pytest.mark.parametrize("form", ["recurrent", "parallel", "chunk1", "chunk2", "chunk3"])
+def test_hand_worked_scalar(form):
+    g = _golden()["scalar"]
+    q, k, v = _seq(g["q"]), _seq(g["k"]), _seq(g["v"])
+    gam = [g["gamma"]]
+    if form == "recurrent":
+        o, s = oracle.recurrent(q, k, v, gam)
+    elif form == "parallel":
+        o, s = oracle.parallel(q, k, v, gam)
+    else:
+        o, s = oracle.chunkwise(q, k, v, gam, int(form[-1]))
+    np.testing.assert_allclose(o[0, 0, :, 0], g["o"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(s[0, 0, 0, 0], g["state"], rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("form", ["recurrent", "parallel", "chunk1", "chunk2"])
+def test_hand_worked_matrix_with_state(form):
+    g = _golden()["matrix_with_state"]
+    q, k, v = _seq(g["q"]), _seq(g["k"]), _seq(g["v"])
+    s0 = np.asarray(g["state_in"], dtype=np.float64)[None, None]
+    gam = [g["gamma"]]
+    if form == "recurrent":
+        o, s = oracle.recurrent(q, k, v, gam, s0)
+    elif form == "parallel":
+        o, s = oracle.parallel(q, k, v, gam, s0)
+    else:
+        o, s = oracle.chunkwise(q, k, v, gam, int(form[-1]), s0)
+    np.testing.assert_allclose(o[0, 0], g["o"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(s[0, 0], g["state"], rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("form", ["recurrent", "parallel", "chunk2"])
+def test_hand_worked_gamma_zero(form):
+    g = _golden()["gamma_zero"]
+    q, k, v = _seq(g["q"]), _seq(g["k"]), _seq(g["v"])
+    gam = [g["gamma"]]
+    if form == "recurrent":
+        o, s = oracle.recurrent(q, k, v, gam)
+    elif form == "parallel":
+        o, s = oracle.parallel(q, k, v, gam)
+    else:
+        o, s = oracle.chunkwise(q, k, v, gam, 2)
+    np.testing.assert_array_equal(o[0, 0], g["o"])
+    np.testing.assert_array_equal(s[0, 0], g["state"])
+
+
+def test_hand_worked_group_norm():
+    g = _golden()["group_norm"]
+    out = oracle.group_norm(np.asarray(g["o"], dtype=np.float64), g["eps"])
+    np.testing.assert_allclose(out, g["out"], rtol=0, atol=1e-15)
+
+
+# --- P2: decay mask against brute force --------------------------------------
+
+@pytest.mark.parametrize("gamma", [0.0, 0.3, 0.5, 0.96875, 1.0 - 2.0 ** -20, 1.0])
+def test_decay_mask_brute_force(gamma):
+    n = 16
+    ref = np.zeros((n, n))
+    for i in range(n):
+        ref[i, i] = 1.0
+        for j in range(i):
+            # D[i, j] = gamma * D[i-1, j]: repeated multiplication
+            ref[i, j] = gamma * ref[i - 1, j]
+    np.testing.assert_allclose(oracle.decay_mask(gamma, n), ref, rtol=1e-14, atol=0)
+    # lower-triangular, unit diagonal ([Medium]: D is lower triangular)
+    assert np.all(np.triu(oracle.decay_mask(gamma, n), 1) == 0)
+
+
+# --- P1 / P9: the three forms agree; state closed form -------------------------
+
+@pytest.mark.parametrize("chunk", [1, 3, 7, 16, 37, 64])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_three_forms_agree(chunk, with_state):
+    rng = np.random.default_rng(11)
+    q, k, v, s0 = _rand(rng, 2, 4, 37, 5, 6, state=with_state)
+    gam = [0.9, 0.5, 0.999, 0.0]
+    o_r, s_r = oracle.recurrent(q, k, v, gam, s0)
+    o_p, s_p = oracle.parallel(q, k, v, gam, s0)
+    o_c, s_c = oracle.chunkwise(q, k, v, gam, chunk, s0)
+    assert oracle.rel_frobenius(o_p, o_r) < 1e-12
+    assert oracle.rel_frobenius(o_c, o_r) < 1e-12
+    assert oracle.rel_frobenius(s_p, s_r) < 1e-12
+    assert oracle.rel_frobenius(s_c, s_r) < 1e-12
+
+
+def test_state_closed_form_brute_force():
+    """S_N = sum_m gamma^(N-1-m) k_m^T v_m + gamma^N S_0, summed term by term."""
+    rng = np.random.default_rng(5)
+    q, k, v, s0 = _rand(rng, 1, 1, 9, 3, 2)
+    g = 0.7
+    ref = g ** 9 * s0[0, 0].copy()
+    for m in range(9):
+        ref += g ** (8 - m) * np.outer(k[0, 0, m], v[0, 0, m])
+    _, s = oracle.recurrent(q, k, v, [g], s0)
+    np.testing.assert_allclose(s[0, 0], ref, rtol=1e-13)
+
+
+# --- P3 / P4: textbook special cases ------------------------------------------
+
+def test_gamma_zero_reduces_to_diagonal():
+    rng = np.random.default_rng(3)
+    q, k, v, _ = _rand(rng, 1, 1, 12, 4, 3, state=False)
+    ref = np.einsum("nk,nk->n", q[0, 0], k[0, 0])[:, None] * v[0, 0]
+    for form in ("recurrent", "parallel", "chunk"):
+        if form == "recurrent":
+            o, _ = oracle.recurrent(q, k, v, [0.0])
+        elif form == "parallel":
+            o, _ = oracle.parallel(q, k, v, [0.0])
+        else:
+            o, _ = oracle.chunkwise(q, k, v, [0.0], 5)
+        np.testing.assert_allclose(o[0, 0], ref, rtol=1e-14, atol=1e-15)
+    # a tiny gamma is a small perturbation of the same result
+    o, _ = oracle.parallel(q, k, v, [1e-12])
+    assert oracle.rel_frobenius(o[0, 0], ref) < 1e-10
+
+
+def test_gamma_one_is_causal_linear_attention():
+    """gamma = 1: o_n = q_n sum_{m<=n} k_m^T v_m (causal linear attention,
+    the link to linear attention on the RetNet blog, Insights)."""
+    rng = np.random.default_rng(4)
+    q, k, v, _ = _rand(rng, 1, 1, 20, 4, 3, state=False)
+    outer = k[0, 0][:, :, None] * v[0, 0][:, None, :]
+    S = np.cumsum(outer, axis=0)
+    ref = np.einsum("nk,nkv->nv", q[0, 0], S)
+    for chunk in (1, 6, 20):
+        o, s = oracle.chunkwise(q, k, v, [1.0], chunk)
+        np.testing.assert_allclose(o[0, 0], ref, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(s[0, 0], S[-1], rtol=1e-12, atol=1e-12)
+
+
+# --- P6: resume from a carried state ------------------------------------------
+
+@pytest.mark.parametrize("split", [1, 13, 32, 49])
+def test_split_sequence_resume(split):
+    rng = np.random.default_rng(6)
+    q, k, v, _ = _rand(rng, 2, 2, 50, 4, 5, state=False)
+    gam = [0.95, 0.6]
+    o_full, s_full = oracle.chunkwise(q, k, v, gam, 8)
+    o1, s1 = oracle.chunkwise(q[:, :, :split], k[:, :, :split], v[:, :, :split], gam, 8)
+    o2, s2 = oracle.chunkwise(q[:, :, split:], k[:, :, split:], v[:, :, split:], gam, 8, s1)
+    assert oracle.rel_frobenius(np.concatenate([o1, o2], axis=2), o_full) < 1e-12
+    assert oracle.rel_frobenius(s2, s_full) < 1e-12
+
+
+def test_step_chain_equals_prefill():
+    """A chunkwise prefill followed by single steps equals one long recurrence."""
+    rng = np.random.default_rng(8)
+    q, k, v, _ = _rand(rng, 2, 3, 30, 4, 4, state=False)
+    gam = [0.9, 0.99, 0.3]
+    o_ref, s_ref = oracle.recurrent(q, k, v, gam)
+    _, s = oracle.chunkwise(q[:, :, :25], k[:, :, :25], v[:, :, :25], gam, 8)
+    for n in range(25, 30):
+        o, s = oracle.step(q[:, :, n], k[:, :, n], v[:, :, n], gam, s)
+        np.testing.assert_allclose(o, o_ref[:, :, n], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(s, s_ref, rtol=1e-12, atol=1e-12)
+
+
+# --- P7: linearity --------------------------------------------------------------
+
+def test_linearity():
+    rng = np.random.default_rng(7)
+    q, k, v, s0 = _rand(rng, 1, 2, 17, 3, 4)
+    v2 = rng.standard_normal(v.shape)
+    s02 = rng.standard_normal(s0.shape)
+    gam = [0.8, 0.97]
+    f = lambda qq, vv, ss: oracle.chunkwise(qq, k, vv, gam, 5, ss)
+    o_a, s_a = f(q, v, s0)
+    o_b, s_b = f(q, v2, s02)
+    o_ab, s_ab = f(q, 2.0 * v - 3.0 * v2, 2.0 * s0 - 3.0 * s02)
+    np.testing.assert_allclose(o_ab, 2 * o_a - 3 * o_b, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(s_ab, 2 * s_a - 3 * s_b, rtol=1e-11, atol=1e-11)
+    o_q, _ = f(2.5 * q, v, s0)
+    np.testing.assert_allclose(o_q, 2.5 * o_a, rtol=1e-12, atol=1e-12)
+
+
+# --- P8: GroupNorm invariants ---------------------------------------------------
+
+def test_group_norm_invariants():
+    rng = np.random.default_rng(9)
+    o = rng.standard_normal((2, 3, 11, 16)) * 3 + 1
+    eps = 1e-5
+    out = oracle.group_norm(o, eps)
+    var = o.var(axis=-1, keepdims=True)
+    np.testing.assert_allclose(out.mean(axis=-1), 0, atol=1e-13)
+    np.testing.assert_allclose(out.var(axis=-1, keepdims=True), var / (var + eps), rtol=1e-12)
+    # shift and positive-scale invariance of each group
+    out2 = oracle.group_norm(4.0 * o + 7.0, 16 * eps)
+    np.testing.assert_allclose(out2, out, rtol=1e-10, atol=1e-12)
+
+
+# --- inputs: bf16 rounding and the decay schedule -------------------------------
+
+def test_bf16_rounding_ties_to_even():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, 1.0 + 2 ** -9, -2.5, 0.0],
+                 dtype=np.float32)
+    got = wl.bf16_bits_to_f64(wl.f32_to_bf16_bits(x))
+    # 1+2^-8 is a tie -> 1 (even); 1+3*2^-8 is a tie -> 1+2^-6 (even); 1+2^-9 -> 1
+    np.testing.assert_array_equal(got, [1.0, 1.0, 1.0 + 2 ** -6, 1.0, -2.5, 0.0])
+
+
+def test_msr_gammas_exact():
+    g = wl.msr_gammas(16)
+    assert g[0] == 0.96875 and g[1] == 0.984375
+    assert float(g[15]) == 1.0 - 2.0 ** -20
+    assert np.all((g > 0) & (g < 1))
+
+
+# --- mutation tests: planted mistakes are caught by the pins --------------------
+
+def _chunkwise_mutant(q, k, v, gammas, chunk, mutation):
+    """A copy of the oracle's chunkwise steps with one planted mistake."""
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    o = np.zeros((B, H, N, dv))
+    R = np.zeros((B, H, dk, dv))
+    for h in range(H):
+        g = gammas[h]
+        for s in range(0, N, chunk):
+            L = min(chunk, N - s)
+            j = np.arange(L)
+            D = oracle.decay_mask(g, L)
+            xi = g ** (j + 1)
+            zeta = g ** (L - 1 - j)
+            if mutation == "xi_exponent":
+                xi = g ** j
+            if mutation == "diag_exclusive":
+                D = D - np.eye(L)
+            for b in range(B):
+                Q, K, V = q[b, h, s:s + L], k[b, h, s:s + L], v[b, h, s:s + L]
+                o[b, h, s:s + L] = ((Q @ K.T) * D) @ V + (Q * xi[:, None]) @ R[b, h]
+                if mutation == "page_chunk_state":   # R_i = K^T V + gamma^chunk R_{i-1}
+                    R[b, h] = g ** L * R[b, h] + K.T @ V
+                elif mutation == "transposed_mask":
+                    pass
+                else:
+                    R[b, h] = g ** L * R[b, h] + K.T @ (V * zeta[:, None])
+            if mutation == "transposed_mask":
+                for b in range(B):
+                    Q, K, V = q[b, h, s:s + L], k[b, h, s:s + L], v[b, h, s:s + L]
+                    o[b, h, s:s + L] = ((Q @ K.T) * D.T) @ V + (Q * xi[:, None]) @ R[b, h]
+                    R[b, h] = g ** L * R[b, h] + K.T @ (V * zeta[:, None])
+    return o, R
+
+
+@pytest.mark.parametrize("mutation", ["xi_exponent", "diag_exclusive", "page_chunk_state",
+                                      "transposed_mask"])
+def test_pins_catch_planted_mistakes(mutation):
+    rng = np.random.default_rng(12)
+    q, k, v, _ = _rand(rng, 1, 2, 24, 3, 3, state=False)
+    gam = [0.9, 0.5]
+    o_ref, s_ref = oracle.recurrent(q, k, v, gam)
+    o_m, s_m = _chunkwise_mutant(q, k, v, gam, 8, mutation)
+    assert oracle.rel_frobenius(o_m, o_ref) > 1e-3 or oracle.rel_frobenius(s_m, s_ref) > 1e-3
+
+
+def test_page_chunk_state_exact_only_for_gamma_one():
+    """The chunk state as printed (no in-chunk decay) equals the recurrence
+    only when gamma = 1; this is why the oracle carries zeta."""
+    rng = np.random.default_rng(13)
+    q, k, v, _ = _rand(rng, 1, 1, 16, 3, 3, state=False)
+    o_ref, s_ref = oracle.recurrent(q, k, v, [1.0])
+    o_m, s_m = _chunkwise_mutant(q, k, v, [1.0], 4, "page_chunk_state")
+    assert oracle.rel_frobenius(o_m, o_ref) < 1e-12
+    assert oracle.rel_frobenius(s_m, s_ref) < 1e-12
