@@ -1,0 +1,131 @@
+/*
+ * retention.h - C ABI of libretention.so: multi-scale retention on NVIDIA
+ * B200 (sm_100a).
+ *
+ * Retention, as defined on the page "RetNet - Retentive Network - A Successor
+ * to Transformer for LLMs" (section Key Equations), has three forms that give
+ * the same output in exact arithmetic:
+ *
+ *   recurrent   S_n = gamma * S_{n-1} + k_n^T v_n,     o_n = q_n S_n
+ *   parallel    O = (Q K^T (.) D) V,   D[n][m] = gamma^(n-m) if n >= m, else 0
+ *   chunkwise   O_[i] = (Q_[i] K_[i]^T (.) D) V_[i] + (Q_[i] (.) xi) R_{i-1}
+ *
+ * with one decay gamma_h per head (multi-scale retention, same page, section
+ * Methods: gamma_h = 1 - 2^(-5-h); here gammas are an input).  The chunk state
+ * is R_i = gamma^L R_{i-1} + K_[i]^T (V_[i] (.) zeta) with xi_j = gamma^(j+1)
+ * and zeta_j = gamma^(L-1-j) for in-chunk position j of a chunk of length L
+ * (the page prints R_i without the in-chunk decay and leaves xi undefined;
+ * these are the readings that make the chunkwise form equal the recurrence).
+ * An optional per-head GroupNorm (same page, Methods: MSR -> GroupNorm)
+ * normalises each (batch, head, token) row of o over its d_v values:
+ * (o - mean) / sqrt(var + eps), biased variance, no affine parameters.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates no memory; scratch space comes from the caller (workspace).
+ *  - Layouts are dense row-major:
+ *        q, k     [B][H][N][dk]        v, o  [B][H][N][dv]
+ *        state    [B][H][dk][dv]  float32 always
+ *        gammas   [H]             float32, each in [0, 1]; values outside give
+ *                                 unspecified (possibly NaN) results
+ *    q, k, v and o share the element type `dtype` (RET_F32 or RET_BF16).
+ *  - q, k, v, o, state and workspace must be 16-byte aligned; dk and dv must be
+ *    multiples of 8.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *    is the legacy default stream).  A return value other than RET_OK means
+ *    that nothing was launched and no memory was written.  Errors raised by a
+ *    kernel while it runs surface on the stream like any CUDA error.
+ *  - Accumulation is float32.  With RET_BF16 inputs the products run on the
+ *    tensor cores with bf16 operands; o is rounded to the input type.
+ */
+#ifndef RETENTION_H_
+#define RETENTION_H_
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define RET_API __attribute__((visibility("default")))
+#else
+#define RET_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { RET_F32 = 0, RET_BF16 = 1 } ret_dtype;
+
+typedef enum {
+  RET_OK = 0,
+  RET_EINVAL = -1,        /* invalid argument: NULL, bad size, misalignment  */
+  RET_EUNSUPPORTED = -2,  /* valid, but no kernel in this build handles it    */
+  RET_ECUDA = -3,         /* a CUDA runtime call failed (ret_last_cuda_error) */
+  RET_EWORKSPACE = -4     /* workspace smaller than the size it must have     */
+} ret_status;
+
+/*
+ * Parallel form, O = (Q K^T (.) D) V, one decay per head; no state enters or
+ * leaves.  ("RetNet - Retentive Network - A Successor to Transformer for
+ * LLMs", Key Equations, Parallel Form; jisaku.com glossary "RetNet",
+ * parallel mode.)
+ *   q, k, v, o : layouts above; N >= 0 (N == 0 writes nothing).
+ *   gn_eps     : < 0 disables the fused GroupNorm, otherwise its epsilon.
+ * Supported: dk, dv in [8, 512]; RET_BF16 runs on the tensor cores when
+ * dk in {64,128,256} and dv in {64,128,256,512}.
+ */
+RET_API int ret_parallel(const void* q, const void* k, const void* v, const float* gammas, void* o,
+                 int B, int H, int N, int dk, int dv, int dtype, float gn_eps, void* stream);
+
+/*
+ * Bytes of workspace ret_chunkwise needs for these sizes (0 if none).  Returns
+ * 0 as well for arguments ret_chunkwise would reject.
+ */
+RET_API size_t ret_chunkwise_workspace(int B, int H, int N, int dk, int dv, int chunk, int dtype);
+
+/*
+ * Chunkwise-recurrent form ("RetNet - Retentive Network - A Successor to
+ * Transformer for LLMs", Key Equations, Chunkwise Recurrent; jisaku.com
+ * glossary "RetNet", chunkwise mode): the sequence is cut into chunks of
+ * `chunk` tokens (the last one may be shorter), each computed in parallel, and
+ * a float32 d_k x d_v state per (batch, head) is carried from chunk to chunk.
+ *   state_in   : initial state [B][H][dk][dv]; NULL means zero.
+ *   state_out  : final state; NULL means not written.  May equal state_in.
+ *   workspace  : device scratch of at least ret_chunkwise_workspace() bytes;
+ *                its contents on entry do not matter; it is overwritten.
+ * The final state is accurate to float32 accumulation (the bf16 path splits
+ * the decayed V operand into two bf16 halves when state_out is requested).
+ * Supported: chunk >= 1 with RET_F32; chunk in {128, 256, 512} for the tensor
+ * core path of RET_BF16, under the same dk/dv rules as ret_parallel.
+ */
+RET_API int ret_chunkwise(const void* q, const void* k, const void* v, const float* gammas, int chunk,
+                  const float* state_in, float* state_out, void* o,
+                  int B, int H, int N, int dk, int dv, int dtype, float gn_eps,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One recurrent decode step for every (batch, head) pair ("RetNet - Retentive
+ * Network - A Successor to Transformer for LLMs", Key Equations, Recurrent
+ * Form):  state <- gamma * state + k^T v,  o = q state  (the updated state).
+ *   q, k  : [B][H][dk]      v, o : [B][H][dv]     (element type dtype)
+ *   state : [B][H][dk][dv] float32, read and written in place.
+ *   gn_eps: < 0 disables the fused GroupNorm of o.
+ * Supported: dk in [8, 4096], dv in [8, 1024].
+ */
+RET_API int ret_step(const void* q, const void* k, const void* v, const float* gammas, float* state,
+             void* o, int B, int H, int dk, int dv, int dtype, float gn_eps, void* stream);
+
+/* Human-readable name of a ret_status value (static storage). */
+RET_API const char* ret_status_string(int status);
+
+/* The cudaError_t of the last call that returned RET_ECUDA in this thread. */
+RET_API int ret_last_cuda_error(void);
+
+/* Library version string (static storage). */
+RET_API const char* ret_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RETENTION_H_ */

@@ -1,1 +1,207 @@
-"""Multi-scale retention on B200: thin Python binding over libretention.so."""
+"""Multi-scale retention on B200: thin Python binding over libretention.so.
+
+Every function here only checks and marshals arguments: it takes torch CUDA
+tensors (PyTorch supplies device memory and the current stream) and calls the
+C ABI declared in include/retention.h.  All arithmetic runs in the library's
+CUDA kernels; there is no CPU or PyTorch fallback.  If the library is missing
+or cannot be loaded the calls raise.
+
+Layouts (row-major, contiguous): q, k [B,H,N,dk]; v, o [B,H,N,dv];
+state [B,H,dk,dv] float32; gammas [H] float32.  q, k, v share one dtype,
+torch.float32 or torch.bfloat16.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libretention.so")
+
+RET_F32, RET_BF16 = 0, 1
+RET_OK, RET_EINVAL, RET_EUNSUPPORTED, RET_ECUDA, RET_EWORKSPACE = 0, -1, -2, -3, -4
+
+# name -> (restype, argtypes) of every symbol include/retention.h declares
+_P, _I, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "ret_parallel": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "ret_chunkwise_workspace": (_S, [_I, _I, _I, _I, _I, _I, _I]),
+    "ret_chunkwise": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _S, _P]),
+    "ret_step": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "ret_status_string": (ctypes.c_char_p, [_I]),
+    "ret_last_cuda_error": (_I, []),
+    "ret_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+class RetentionError(RuntimeError):
+    def __init__(self, fn: str, status: int, detail: str = ""):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_string(status)} ({status}){detail}")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libretention.so (once) and bind every exported symbol."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m linear_recurrent_sequence_scale_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().ret_status_string(status).decode()
+
+
+def version() -> str:
+    return load_library().ret_version().decode()
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return RET_F32
+    if t.dtype == torch.bfloat16:
+        return RET_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _check(t, name, dtype=None, shape=None, device=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    torch = _torch()
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _raise(fn, status):
+    lib = load_library()
+    detail = f", cudaError {lib.ret_last_cuda_error()}" if status == RET_ECUDA else ""
+    raise RetentionError(fn, status, detail)
+
+
+def _seq_args(q, k, v, gammas):
+    torch = _torch()
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B,H,N,d]")
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _check(q, "q", device=dev)
+    _check(k, "k", dtype=q.dtype, shape=(B, H, N, dk), device=dev)
+    _check(v, "v", dtype=q.dtype, shape=(B, H, N, dv), device=dev)
+    _check(gammas, "gammas", dtype=torch.float32, shape=(H,), device=dev)
+    return B, H, N, dk, dv, dev
+
+
+def parallel(q, k, v, gammas, gn_eps=None, out=None):
+    """Parallel form O = (Q K^T (.) D) V (ret_parallel); returns o."""
+    torch = _torch()
+    B, H, N, dk, dv, dev = _seq_args(q, k, v, gammas)
+    if out is None:
+        out = torch.empty((B, H, N, dv), dtype=q.dtype, device=dev)
+    _check(out, "out", dtype=q.dtype, shape=(B, H, N, dv), device=dev)
+    eps = -1.0 if gn_eps is None else float(gn_eps)
+    s = load_library().ret_parallel(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), _ptr(out),
+                                    B, H, N, dk, dv, _dtype_code(q), eps, _stream(dev))
+    if s != RET_OK:
+        _raise("ret_parallel", s)
+    return out
+
+
+def chunkwise_workspace_bytes(B, H, N, dk, dv, chunk, dtype) -> int:
+    torch = _torch()
+    code = RET_BF16 if dtype == torch.bfloat16 else RET_F32
+    return int(load_library().ret_chunkwise_workspace(B, H, N, dk, dv, chunk, code))
+
+
+def chunkwise(q, k, v, gammas, chunk, state_in=None, state_out=None, return_state=False,
+              gn_eps=None, out=None, workspace=None):
+    """Chunkwise-recurrent form (ret_chunkwise).
+
+    Returns o, or (o, state) when return_state is True or state_out is given.
+    state_out may be the same tensor as state_in (updated in place).
+    workspace: optional uint8 CUDA tensor of at least chunkwise_workspace_bytes().
+    """
+    torch = _torch()
+    B, H, N, dk, dv, dev = _seq_args(q, k, v, gammas)
+    sshape = (B, H, dk, dv)
+    if state_in is not None:
+        _check(state_in, "state_in", dtype=torch.float32, shape=sshape, device=dev)
+    if state_out is None and return_state:
+        state_out = torch.empty(sshape, dtype=torch.float32, device=dev)
+    if state_out is not None:
+        _check(state_out, "state_out", dtype=torch.float32, shape=sshape, device=dev)
+    if out is None:
+        out = torch.empty((B, H, N, dv), dtype=q.dtype, device=dev)
+    _check(out, "out", dtype=q.dtype, shape=(B, H, N, dv), device=dev)
+    need = chunkwise_workspace_bytes(B, H, N, dk, dv, chunk, q.dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0
+    if workspace is not None:
+        _check(workspace, "workspace", device=dev)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    eps = -1.0 if gn_eps is None else float(gn_eps)
+    s = load_library().ret_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), int(chunk),
+                                     _ptr(state_in), _ptr(state_out), _ptr(out),
+                                     B, H, N, dk, dv, _dtype_code(q), eps,
+                                     _ptr(workspace), ws_bytes, _stream(dev))
+    if s != RET_OK:
+        _raise("ret_chunkwise", s)
+    if state_out is not None:
+        return out, state_out
+    return out
+
+
+def step(q, k, v, gammas, state, gn_eps=None, out=None):
+    """One recurrent decode step (ret_step): state is updated in place; returns o.
+    q, k [B,H,dk]; v [B,H,dv]; state [B,H,dk,dv] float32."""
+    torch = _torch()
+    if q.dim() != 3:
+        raise ValueError("q, k, v must be [B,H,d] for a decode step")
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    _check(q, "q", device=dev)
+    _check(k, "k", dtype=q.dtype, shape=(B, H, dk), device=dev)
+    _check(v, "v", dtype=q.dtype, shape=(B, H, dv), device=dev)
+    _check(gammas, "gammas", dtype=torch.float32, shape=(H,), device=dev)
+    _check(state, "state", dtype=torch.float32, shape=(B, H, dk, dv), device=dev)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=dev)
+    _check(out, "out", dtype=q.dtype, shape=(B, H, dv), device=dev)
+    eps = -1.0 if gn_eps is None else float(gn_eps)
+    s = load_library().ret_step(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), _ptr(state), _ptr(out),
+                                B, H, dk, dv, _dtype_code(q), eps, _stream(dev))
+    if s != RET_OK:
+        _raise("ret_step", s)
+    return out

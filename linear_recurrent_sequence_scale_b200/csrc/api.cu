@@ -1,0 +1,122 @@
+// C ABI of libretention.so: argument checks and kernel dispatch.
+//
+// Every check runs on the host before anything is launched, so a non-zero
+// status means no kernel ran and no memory was touched.
+#include <math.h>
+#include <stdint.h>
+
+#include "kernels.h"
+#include "retention.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return RET_OK;
+  g_last_cuda_error = static_cast<int>(e);
+  return RET_ECUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_dtype(int dt) { return dt == RET_F32 || dt == RET_BF16; }
+
+// Sizes shared by the sequence forms.  dk, dv: multiples of 8 in [8, 512].
+int check_seq_dims(int B, int H, int N, int dk, int dv, int dtype) {
+  if (B < 1 || H < 1 || N < 0 || dk < 8 || dv < 8) return RET_EINVAL;
+  if (dk % 8 || dv % 8) return RET_EINVAL;
+  if (!valid_dtype(dtype)) return RET_EINVAL;
+  if ((int64_t)B * H > 65535) return RET_EUNSUPPORTED;
+  if (dk > 512 || dv > 512) return RET_EUNSUPPORTED;
+  if ((int64_t)B * H * N * (dk > dv ? dk : dv) > ((int64_t)1 << 40)) return RET_EUNSUPPORTED;
+  return RET_OK;
+}
+
+int check_eps(float eps) { return isnan(eps) ? RET_EINVAL : RET_OK; }
+
+}  // namespace
+
+extern "C" {
+
+const char* ret_status_string(int status) {
+  switch (status) {
+    case RET_OK: return "ok";
+    case RET_EINVAL: return "invalid argument";
+    case RET_EUNSUPPORTED: return "unsupported configuration";
+    case RET_ECUDA: return "CUDA runtime error";
+    case RET_EWORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+int ret_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* ret_version(void) { return "retention-b200 0.1 (sm_100a)"; }
+
+int ret_parallel(const void* q, const void* k, const void* v, const float* gammas, void* o,
+                 int B, int H, int N, int dk, int dv, int dtype, float gn_eps, void* stream) {
+  int s = check_seq_dims(B, H, N, dk, dv, dtype);
+  if (s) return s;
+  if ((s = check_eps(gn_eps))) return s;
+  if (N == 0) return RET_OK;
+  if (!q || !k || !v || !o || !gammas) return RET_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(ret::launch_simt_parallel(q, k, v, gammas, o, B, H, N, dk, dv, dtype,
+                                               gn_eps, st));
+}
+
+size_t ret_chunkwise_workspace(int B, int H, int N, int dk, int dv, int chunk, int dtype) {
+  if (check_seq_dims(B, H, N, dk, dv, dtype) != RET_OK || chunk < 1) return 0;
+  if (N == 0) return 0;
+  return ret::simt_workspace_bytes(B, H, N, dk, dv, chunk);
+}
+
+int ret_chunkwise(const void* q, const void* k, const void* v, const float* gammas, int chunk,
+                  const float* state_in, float* state_out, void* o, int B, int H, int N, int dk,
+                  int dv, int dtype, float gn_eps, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  int s = check_seq_dims(B, H, N, dk, dv, dtype);
+  if (s) return s;
+  if ((s = check_eps(gn_eps))) return s;
+  if (chunk < 1) return RET_EINVAL;
+  if (!gammas) return RET_EINVAL;
+  if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
+    return RET_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t state_bytes = sizeof(float) * (size_t)B * H * dk * dv;
+  if (N == 0) {
+    // No tokens: the final state is the initial one.
+    if (!state_out) return RET_OK;
+    if (state_in == state_out) return RET_OK;
+    if (state_in)
+      return cuda_status(
+          cudaMemcpyAsync(state_out, state_in, state_bytes, cudaMemcpyDeviceToDevice, st));
+    return cuda_status(cudaMemsetAsync(state_out, 0, state_bytes, st));
+  }
+  if (!q || !k || !v || !o) return RET_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_EINVAL;
+  const size_t need = ret_chunkwise_workspace(B, H, N, dk, dv, chunk, dtype);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return RET_EWORKSPACE;
+  if (workspace && !aligned16(workspace)) return RET_EINVAL;
+  return cuda_status(ret::launch_simt_chunkwise(q, k, v, gammas, chunk, state_in, state_out, o,
+                                                B, H, N, dk, dv, dtype, gn_eps, workspace, st));
+}
+
+int ret_step(const void* q, const void* k, const void* v, const float* gammas, float* state,
+             void* o, int B, int H, int dk, int dv, int dtype, float gn_eps, void* stream) {
+  if (B < 1 || H < 1 || dk < 8 || dv < 8 || dk % 8 || dv % 8) return RET_EINVAL;
+  if (!valid_dtype(dtype)) return RET_EINVAL;
+  int s = check_eps(gn_eps);
+  if (s) return s;
+  if (dk > 4096 || dv > 1024 || (int64_t)B * H > 65535) return RET_EUNSUPPORTED;
+  if (!q || !k || !v || !gammas || !state || !o) return RET_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(o))
+    return RET_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(
+      ret::launch_step(q, k, v, gammas, state, o, B, H, dk, dv, dtype, gn_eps, st));
+}
+
+}  // extern "C"

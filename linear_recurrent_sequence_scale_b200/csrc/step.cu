@@ -1,0 +1,183 @@
+// Recurrent decode step: state <- gamma*state + k^T v, o = q state.
+//
+// "RetNet - Retentive Network - A Successor to Transformer for LLMs", Key
+// Equations, Recurrent Form.  Per (batch, head) the float32 state is a
+// dk x dv row-major matrix; one step reads and writes all of it once, so the
+// kernel is bound by HBM bandwidth (about 0.5 flop per byte).
+//
+// Mapping: a CTA owns STEP_COLS = 128 state columns of one (b, h) and all dk
+// rows.  Each warp covers the 128 columns of a row with one 16-byte access per
+// lane (fully coalesced 512-byte rows); the 8 warps split the rows, each
+// keeping STEP_UNROLL independent row loads in flight before it updates and
+// stores them.  The partial q.S sums of the 8 warps meet in shared memory.
+// With GroupNorm the CTAs of one (b, h) form a thread-block cluster and
+// exchange their row statistics through distributed shared memory.
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace ret {
+
+constexpr int STEP_COLS = 128;
+constexpr int STEP_THREADS = 256;
+constexpr int STEP_RG = STEP_THREADS / (STEP_COLS / 4);  // 8 row groups (= warps)
+constexpr int STEP_UNROLL = 8;
+
+__device__ __forceinline__ float block_sum_256(float x, float* scratch /* >= 8 floats */) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  const int w = threadIdx.x >> 5;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) scratch[w] = x;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < STEP_THREADS / 32; ++i) t += scratch[i];
+  return t;
+}
+
+template <typename T, bool GN>
+__global__ void __launch_bounds__(STEP_THREADS)
+step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+            const float* __restrict__ gammas, float* __restrict__ state, T* __restrict__ o,
+            int H, int dk, int dv, float eps) {
+  extern __shared__ float smem[];
+  float* qs = smem;                       // [dk]
+  float* ks = smem + dk;                  // [dk]
+  float* red = smem + 2 * dk;             // [STEP_RG][STEP_COLS]
+  __shared__ float scratch[8];
+  __shared__ float stats[2];              // this CTA's partial sum, sum of squares
+
+  const int bh = blockIdx.y;
+  const int h = bh % H;
+  const int c0 = blockIdx.x * STEP_COLS;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int rg = tid >> 5;
+
+  for (int i = tid; i < dk; i += STEP_THREADS) {
+    qs[i] = Elem<T>::ld(q + (size_t)bh * dk + i);
+    ks[i] = Elem<T>::ld(k + (size_t)bh * dk + i);
+  }
+  const float g = gammas[h];
+  const int c = c0 + 4 * lane;
+  const bool cval = c < dv;  // dv is a multiple of 4, so c..c+3 are all valid
+  float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (cval) vv = Elem<T>::ld4(v + (size_t)bh * dv + c);
+  __syncthreads();
+
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float* S = state + (size_t)bh * dk * dv + c;
+  for (int r0 = rg; r0 < dk; r0 += STEP_RG * STEP_UNROLL) {
+    float4 s[STEP_UNROLL];
+#pragma unroll
+    for (int u = 0; u < STEP_UNROLL; ++u) {
+      const int r = r0 + u * STEP_RG;
+      if (cval && r < dk) s[u] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)r * dv));
+    }
+#pragma unroll
+    for (int u = 0; u < STEP_UNROLL; ++u) {
+      const int r = r0 + u * STEP_RG;
+      if (cval && r < dk) {
+        const float kr = ks[r], qr = qs[r];
+        float4 t;
+        t.x = fmaf(kr, vv.x, g * s[u].x);
+        t.y = fmaf(kr, vv.y, g * s[u].y);
+        t.z = fmaf(kr, vv.z, g * s[u].z);
+        t.w = fmaf(kr, vv.w, g * s[u].w);
+        __stcs(reinterpret_cast<float4*>(S + (size_t)r * dv), t);
+        acc.x = fmaf(qr, t.x, acc.x);
+        acc.y = fmaf(qr, t.y, acc.y);
+        acc.z = fmaf(qr, t.z, acc.z);
+        acc.w = fmaf(qr, t.w, acc.w);
+      }
+    }
+  }
+  red[rg * STEP_COLS + 4 * lane + 0] = acc.x;
+  red[rg * STEP_COLS + 4 * lane + 1] = acc.y;
+  red[rg * STEP_COLS + 4 * lane + 2] = acc.z;
+  red[rg * STEP_COLS + 4 * lane + 3] = acc.w;
+  __syncthreads();
+
+  const int oc = c0 + tid;
+  const bool oval = tid < STEP_COLS && oc < dv;
+  float val = 0.f;
+  if (tid < STEP_COLS) {
+#pragma unroll
+    for (int i = 0; i < STEP_RG; ++i) val += red[i * STEP_COLS + tid];
+  }
+  if constexpr (GN) {
+    cg::cluster_group cluster = cg::this_cluster();
+    const unsigned nblk = cluster.num_blocks();
+    float part = block_sum_256(oval ? val : 0.f, scratch);
+    if (tid == 0) stats[0] = part;
+    cluster.sync();
+    float tot = 0.f;
+    for (unsigned r = 0; r < nblk; ++r) tot += cluster.map_shared_rank(stats, r)[0];
+    const float mean = tot / static_cast<float>(dv);
+    const float dev = oval ? val - mean : 0.f;
+    part = block_sum_256(dev * dev, scratch);
+    if (tid == 0) stats[1] = part;
+    cluster.sync();
+    float sq = 0.f;
+    for (unsigned r = 0; r < nblk; ++r) sq += cluster.map_shared_rank(stats, r)[1];
+    const float inv = 1.0f / sqrtf(sq / static_cast<float>(dv) + eps);
+    if (oval) Elem<T>::st(o + (size_t)bh * dv + oc, dev * inv);
+    cluster.sync();  // peers may still be reading this CTA's stats
+  } else {
+    if (oval) Elem<T>::st(o + (size_t)bh * dv + oc, val);
+  }
+}
+
+template <typename T>
+static cudaError_t launch_step_t(const void* q, const void* k, const void* v, const float* gammas,
+                                 float* state, void* o, int B, int H, int dk, int dv, float eps,
+                                 cudaStream_t st) {
+  const int nct = cdiv(dv, STEP_COLS);
+  dim3 grid(nct, B * H);
+  const size_t smem = sizeof(float) * (2 * dk + STEP_RG * STEP_COLS);
+  const T* qq = static_cast<const T*>(q);
+  const T* kk = static_cast<const T*>(k);
+  const T* vv = static_cast<const T*>(v);
+  T* oo = static_cast<T*>(o);
+  if (eps < 0.f) {
+    auto fn = step_kernel<T, false>;
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    fn<<<grid, STEP_THREADS, smem, st>>>(qq, kk, vv, gammas, state, oo, H, dk, dv, eps);
+    return cudaPeekAtLastError();
+  }
+  auto fn = step_kernel<T, true>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(STEP_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nct;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, fn, qq, kk, vv, gammas, state, oo, H, dk, dv, eps);
+}
+
+cudaError_t launch_step(const void* q, const void* k, const void* v, const float* gammas,
+                        float* state, void* o, int B, int H, int dk, int dv, int dtype,
+                        float eps, cudaStream_t st) {
+  if (dtype == RET_BF16)
+    return launch_step_t<__nv_bfloat16>(q, k, v, gammas, state, o, B, H, dk, dv, eps, st);
+  return launch_step_t<float>(q, k, v, gammas, state, o, B, H, dk, dv, eps, st);
+}
+
+}  // namespace ret

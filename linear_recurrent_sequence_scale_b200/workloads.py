@@ -141,3 +141,22 @@ def make_decode_token(w: Workload, step: int):
     k = draw(rng, (w.B, w.H, w.dk), s, w.dtype)
     v = draw(rng, (w.B, w.H, w.dv), s, w.dtype)
     return q, k, v
+
+
+def to_torch(t: Tensor, device="cuda", pin=False):
+    """Move a stored input to torch without changing a bit: float32 stays
+    float32, bf16 bit patterns become torch.bfloat16."""
+    import torch
+    if t.dtype == "f32":
+        x = torch.from_numpy(np.ascontiguousarray(t.store))
+    else:
+        x = torch.from_numpy(np.ascontiguousarray(t.store).view(np.int16)).view(torch.bfloat16)
+    if pin:
+        return x.pin_memory()
+    return x.to(device)
+
+
+def from_torch(x) -> np.ndarray:
+    """A torch tensor (any device, float32 or bf16) as float64 numpy."""
+    import torch
+    return x.detach().to(device="cpu", dtype=torch.float64).numpy()

@@ -1,0 +1,112 @@
+"""The C ABI without a GPU: the library loads, exports every symbol the header
+declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_recurrent_sequence_scale_b200 as ret
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "retention.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"RET_API\s+[\w\s\*]*?\b(ret_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(ret.LIB_PATH):
+        from linear_recurrent_sequence_scale_b200 import build
+        build.build()
+    return ret.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("ret_parallel", "ret_chunkwise", "ret_chunkwise_workspace", "ret_step",
+              "ret_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(ret.LIB_PATH)
+    for name in _declared():
+        assert hasattr(raw, name), name
+    assert set(_declared()) <= set(ret.SIGNATURES)
+
+
+def test_status_strings(lib):
+    assert lib.ret_status_string(0) == b"ok"
+    assert lib.ret_status_string(-1) == b"invalid argument"
+    assert lib.ret_status_string(-2) == b"unsupported configuration"
+    assert lib.ret_status_string(-3) == b"CUDA runtime error"
+    assert lib.ret_status_string(-4) == b"workspace too small"
+    assert b"sm_100a" in lib.ret_version()
+
+
+P = ctypes.c_void_p
+A = P(0x10000)         # a 16-byte aligned fake address: never dereferenced,
+M = P(0x10008)         # every call below is rejected before any launch
+
+
+def test_parallel_rejects_bad_arguments(lib):
+    f = lib.ret_parallel
+    ok = dict(B=1, H=2, N=16, dk=64, dv=64, dt=1, eps=-1.0)
+
+    def call(q=A, k=A, v=A, g=A, o=A, **kw):
+        a = {**ok, **kw}
+        return f(q, k, v, g, o, a["B"], a["H"], a["N"], a["dk"], a["dv"], a["dt"], a["eps"], None)
+
+    assert call(q=None) == ret.RET_EINVAL
+    assert call(g=None) == ret.RET_EINVAL
+    assert call(o=M) == ret.RET_EINVAL            # misaligned
+    assert call(B=0) == ret.RET_EINVAL
+    assert call(dk=60) == ret.RET_EINVAL          # not a multiple of 8
+    assert call(dv=0) == ret.RET_EINVAL
+    assert call(dt=7) == ret.RET_EINVAL
+    assert call(eps=float("nan")) == ret.RET_EINVAL
+    assert call(dk=1024) == ret.RET_EUNSUPPORTED
+    assert call(B=1000, H=1000) == ret.RET_EUNSUPPORTED
+    # an empty sequence is valid and writes nothing
+    assert call(N=0, q=None, k=None, v=None, o=None) == ret.RET_OK
+
+
+def test_chunkwise_rejects_bad_arguments(lib):
+    f = lib.ret_chunkwise
+    need = lib.ret_chunkwise_workspace(1, 2, 300, 64, 64, 64, 0)
+    assert need > 0
+    assert lib.ret_chunkwise_workspace(1, 2, 300, 64, 64, 0, 0) == 0   # invalid chunk
+
+    def call(q=A, k=A, v=A, g=A, chunk=64, si=None, so=None, o=A, N=300, dt=0, ws=A,
+             wsb=None, eps=-1.0):
+        wsb = need if wsb is None else wsb
+        return f(q, k, v, g, chunk, si, so, o, 1, 2, N, 64, 64, dt, eps, ws, wsb, None)
+
+    assert call(chunk=0) == ret.RET_EINVAL
+    assert call(g=None) == ret.RET_EINVAL
+    assert call(si=M) == ret.RET_EINVAL
+    assert call(v=None) == ret.RET_EINVAL
+    assert call(ws=None) == ret.RET_EWORKSPACE
+    assert call(wsb=need - 1) == ret.RET_EWORKSPACE
+    assert call(ws=M) == ret.RET_EINVAL
+    assert call(N=-1) == ret.RET_EINVAL
+    # no tokens, no state requested: nothing to do
+    assert call(N=0, q=None, k=None, v=None, o=None, ws=None, wsb=0) == ret.RET_OK
+
+
+def test_step_rejects_bad_arguments(lib):
+    f = lib.ret_step
+
+    def call(q=A, k=A, v=A, g=A, s=A, o=A, B=2, H=2, dk=64, dv=64, dt=1, eps=-1.0):
+        return f(q, k, v, g, s, o, B, H, dk, dv, dt, eps, None)
+
+    assert call(s=None) == ret.RET_EINVAL
+    assert call(s=M) == ret.RET_EINVAL
+    assert call(dk=12) == ret.RET_EINVAL
+    assert call(dv=2048) == ret.RET_EUNSUPPORTED
+    assert call(dt=-1) == ret.RET_EINVAL
+    assert call(eps=float("nan")) == ret.RET_EINVAL

@@ -1,0 +1,232 @@
+"""CUDA path against the CPU oracle, element by element on the same inputs.
+
+Tolerances (rel-Frobenius over the whole output): 1e-5 for float32 inputs,
+2e-2 for bf16 inputs with float32 accumulation, 1e-4 for every float32 state
+returned.  bf16 inputs are rounded once by the input generator and the oracle
+consumes exactly those rounded values in float64.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from linear_recurrent_sequence_scale_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "bf16": 2e-2}
+STATE_TOL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch
+
+
+@pytest.fixture(scope="module")
+def ret(torch_cuda):
+    import linear_recurrent_sequence_scale_b200 as ret
+    ret.load_library()
+    return ret
+
+
+def _dev(t):
+    return wl.to_torch(t, "cuda")
+
+
+def _gam(torch, g):
+    return torch.from_numpy(np.asarray(g, dtype=np.float32)).cuda()
+
+
+def _rel(x, ref):
+    return oracle.rel_frobenius(wl.from_torch(x) if not isinstance(x, np.ndarray) else x, ref)
+
+
+def _ref_chunkwise(inp, chunk, gn, with_state_in):
+    s0 = inp["state"].exact if with_state_in else None
+    o, s = oracle.chunkwise(inp["q"].exact, inp["k"].exact, inp["v"].exact, inp["gammas"],
+                            chunk, s0)
+    if gn is not None:
+        o = oracle.group_norm(o, gn)
+    return o, s
+
+
+# --- the tiny float32 workload: all three forms ---------------------------------
+
+def test_tiny_f32_all_three_forms(torch_cuda, ret):
+    torch = torch_cuda
+    w = wl.WORKLOADS["tiny_f32"]
+    inp = wl.make_inputs(w.B, w.H, w.N, w.dk, w.dv, "f32", seed=w.seed)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    o_ref, s_ref = oracle.recurrent(inp["q"].exact, inp["k"].exact, inp["v"].exact, inp["gammas"])
+
+    o_par = ret.parallel(q, k, v, g)
+    o_chk, s_chk = ret.chunkwise(q, k, v, g, w.chunk, return_state=True)
+    state = torch.zeros((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device="cuda")
+    o_rec = torch.empty_like(v)
+    for n in range(w.N):
+        o_rec[:, :, n] = ret.step(q[:, :, n].contiguous(), k[:, :, n].contiguous(),
+                                  v[:, :, n].contiguous(), g, state)
+    torch.cuda.synchronize()
+    assert _rel(o_par, o_ref) <= TOL["f32"]
+    assert _rel(o_chk, o_ref) <= TOL["f32"]
+    assert _rel(o_rec, o_ref) <= TOL["f32"]
+    assert _rel(s_chk, s_ref) <= STATE_TOL
+    assert _rel(state, s_ref) <= STATE_TOL
+
+
+# --- chunkwise: several tiles, ragged tails, GroupNorm, carried state ------------
+
+CHUNK_CASES = [
+    # dtype, B, H, N, dk, dv, chunk, gn_eps, state_in
+    ("bf16", 1, 3, 1000, 256, 512, 512, 1e-5, True),
+    ("bf16", 2, 2, 700, 256, 256, 128, None, False),
+    ("bf16", 1, 4, 333, 64, 64, 128, None, True),
+    ("bf16", 2, 2, 640, 128, 128, 256, 1e-5, False),
+    ("bf16", 1, 2, 1100, 128, 512, 256, None, True),
+    ("f32", 1, 3, 301, 128, 64, 37, None, True),
+    ("f32", 2, 2, 200, 64, 96, 64, 1e-5, False),
+    ("f32", 1, 2, 130, 32, 40, 1, None, True),
+]
+
+
+@pytest.mark.parametrize("case", CHUNK_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_chunkwise_parity(torch_cuda, ret, case):
+    torch = torch_cuda
+    dt, B, H, N, dk, dv, chunk, gn, with_s0 = case
+    inp = wl.make_inputs(B, H, N, dk, dv, dt, seed=100 + N, with_state=with_s0)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    s0 = _dev(inp["state"]) if with_s0 else None
+    o, s = ret.chunkwise(q, k, v, g, chunk, state_in=s0, return_state=True, gn_eps=gn)
+    torch.cuda.synchronize()
+    o_ref, s_ref = _ref_chunkwise(inp, chunk, gn, with_s0)
+    assert _rel(o, o_ref) <= TOL[dt]
+    assert _rel(s, s_ref) <= STATE_TOL
+
+
+def test_chunkwise_without_state_out_and_in_place(torch_cuda, ret):
+    torch = torch_cuda
+    B, H, N, dk, dv, C = 1, 2, 520, 128, 128, 128
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=7, with_state=True)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    o_ref, s_ref = _ref_chunkwise(inp, C, None, True)
+    o1 = ret.chunkwise(q, k, v, g, C, state_in=_dev(inp["state"]))
+    s = _dev(inp["state"])
+    o2, s2 = ret.chunkwise(q, k, v, g, C, state_in=s, state_out=s)   # in place
+    torch.cuda.synchronize()
+    assert s2.data_ptr() == s.data_ptr()
+    assert _rel(o1, o_ref) <= TOL["bf16"]
+    assert _rel(o2, o_ref) <= TOL["bf16"]
+    assert _rel(s, s_ref) <= STATE_TOL
+
+
+# --- parallel form -----------------------------------------------------------------
+
+PAR_CASES = [
+    ("bf16", 2, 2, 777, 128, 128, None),
+    ("bf16", 1, 2, 512, 256, 512, 1e-5),
+    ("bf16", 1, 3, 300, 64, 256, None),
+    ("f32", 1, 2, 257, 64, 64, 1e-5),
+]
+
+
+@pytest.mark.parametrize("case", PAR_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_parallel_parity(torch_cuda, ret, case):
+    torch = torch_cuda
+    dt, B, H, N, dk, dv, gn = case
+    inp = wl.make_inputs(B, H, N, dk, dv, dt, seed=200 + N)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    o = ret.parallel(q, k, v, _gam(torch, inp["gammas"]), gn_eps=gn)
+    torch.cuda.synchronize()
+    o_ref, _ = oracle.parallel(inp["q"].exact, inp["k"].exact, inp["v"].exact, inp["gammas"])
+    if gn is not None:
+        o_ref = oracle.group_norm(o_ref, gn)
+    assert _rel(o, o_ref) <= TOL[dt]
+
+
+# --- decode step -------------------------------------------------------------------
+
+STEP_CASES = [
+    ("bf16", 2, 3, 256, 512, None),
+    ("bf16", 2, 3, 256, 512, 1e-5),
+    ("f32", 3, 2, 64, 64, None),
+    ("f32", 1, 2, 136, 200, 1e-5),
+    ("bf16", 1, 1, 8, 1024, 1e-5),
+]
+
+
+@pytest.mark.parametrize("case", STEP_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_step_parity(torch_cuda, ret, case):
+    torch = torch_cuda
+    dt, B, H, dk, dv, gn = case
+    T = 5
+    inp = wl.make_inputs(B, H, T, dk, dv, dt, seed=300 + dk, with_state=True)
+    state = _dev(inp["state"])
+    S = inp["state"].exact
+    for n in range(T):
+        qn, kn, vn = (inp[x].exact[:, :, n] for x in ("q", "k", "v"))
+        o_ref, S = oracle.step(qn, kn, vn, inp["gammas"], S)
+        if gn is not None:
+            o_ref = oracle.group_norm(o_ref, gn)
+        o = ret.step(_dev(inp["q"])[:, :, n].contiguous(), _dev(inp["k"])[:, :, n].contiguous(),
+                     _dev(inp["v"])[:, :, n].contiguous(), _gam(torch, inp["gammas"]), state,
+                     gn_eps=gn)
+        torch.cuda.synchronize()
+        assert _rel(o, o_ref) <= TOL[dt]
+    assert _rel(state, S) <= STATE_TOL
+
+
+# --- degenerate cases --------------------------------------------------------------
+
+@pytest.mark.parametrize("dt", ["bf16", "f32"])
+def test_gamma_zero_and_one(torch_cuda, ret, dt):
+    """gamma = 0 reduces to o_n = (q_n.k_n) v_n; gamma = 1 is causal linear
+    attention; both must stay finite (no 0*log(0) NaN)."""
+    torch = torch_cuda
+    B, H, N, dk, dv, C = 1, 2, 300, 64, 64, 128
+    inp = wl.make_inputs(B, H, N, dk, dv, dt, seed=9, gammas=[0.0, 1.0])
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    o_ref, s_ref = oracle.chunkwise(inp["q"].exact, inp["k"].exact, inp["v"].exact,
+                                    inp["gammas"], C)
+    o, s = ret.chunkwise(q, k, v, g, C, return_state=True)
+    op = ret.parallel(q, k, v, g)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o.float()).all() and torch.isfinite(op.float()).all()
+    assert _rel(o, o_ref) <= TOL[dt]
+    assert _rel(op, o_ref) <= TOL[dt]
+    assert _rel(s, s_ref) <= STATE_TOL
+
+
+def test_single_token_and_short_sequence(torch_cuda, ret):
+    torch = torch_cuda
+    for N in (1, 5, 127, 129):
+        inp = wl.make_inputs(1, 2, N, 128, 128, "bf16", seed=N, with_state=True)
+        q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+        g = _gam(torch, inp["gammas"])
+        o, s = ret.chunkwise(q, k, v, g, 256, state_in=_dev(inp["state"]), return_state=True)
+        torch.cuda.synchronize()
+        o_ref, s_ref = _ref_chunkwise(inp, 256, None, True)
+        assert _rel(o, o_ref) <= TOL["bf16"], N
+        assert _rel(s, s_ref) <= STATE_TOL, N
+
+
+def test_empty_sequence_copies_state(torch_cuda, ret):
+    torch = torch_cuda
+    B, H, dk, dv = 1, 2, 64, 64
+    q = torch.empty((B, H, 0, dk), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty((B, H, 0, dv), dtype=torch.bfloat16, device="cuda")
+    g = _gam(torch, [0.9, 0.5])
+    s0 = torch.randn((B, H, dk, dv), device="cuda")
+    o, s = ret.chunkwise(q, q, v, g, 128, state_in=s0, return_state=True)
+    o2, z = ret.chunkwise(q, q, v, g, 128, return_state=True)
+    op = ret.parallel(q, q, v, g)
+    torch.cuda.synchronize()
+    assert o.numel() == 0 and op.numel() == 0
+    assert torch.equal(s, s0)
+    assert torch.count_nonzero(z) == 0
