@@ -121,6 +121,14 @@ RET_API const char* ret_status_string(int status);
 /* The cudaError_t of the last call that returned RET_ECUDA in this thread. */
 RET_API int ret_last_cuda_error(void);
 
+/*
+ * Reads and clears the flag the tensor-core kernels set when one of their
+ * bounded waits on an mbarrier ran out (a protocol failure that would
+ * otherwise hang the GPU): 0 if none, otherwise the code of the wait site, -1
+ * if the flag could not be read.  Synchronous with respect to the device.
+ */
+RET_API int ret_device_error(void);
+
 /* Library version string (static storage). */
 RET_API const char* ret_version(void);
 

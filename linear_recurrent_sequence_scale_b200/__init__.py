@@ -30,6 +30,7 @@ SIGNATURES = {
     "ret_status_string": (ctypes.c_char_p, [_I]),
     "ret_last_cuda_error": (_I, []),
     "ret_version": (ctypes.c_char_p, []),
+    "ret_device_error": (_I, []),
 }
 
 _lib = None
@@ -60,6 +61,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 def status_string(status: int) -> str:
     return load_library().ret_status_string(status).decode()
+
+
+def device_error() -> int:
+    """Read and clear the tensor-core kernels' timed-out-wait flag (0 = none)."""
+    return int(load_library().ret_device_error())
 
 
 def version() -> str:

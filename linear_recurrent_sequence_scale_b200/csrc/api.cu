@@ -35,6 +35,17 @@ int check_seq_dims(int B, int H, int N, int dk, int dv, int dtype) {
 
 int check_eps(float eps) { return isnan(eps) ? RET_EINVAL : RET_OK; }
 
+bool pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1)) == 0; }
+
+// Shapes the tensor-core kernels handle (bf16 only).
+bool tc_dims(int dk, int dv) { return pow2_in(dk, 64, 256) && pow2_in(dv, 64, 512); }
+bool tc_chunk(int chunk) { return pow2_in(chunk, 128, 512); }
+
+size_t tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk) {
+  const size_t nc = (size_t)((N + chunk - 1) / chunk);
+  return 2 * (size_t)B * H * nc * dk * dv;
+}
+
 }  // namespace
 
 extern "C" {
@@ -54,6 +65,13 @@ int ret_last_cuda_error(void) { return g_last_cuda_error; }
 
 const char* ret_version(void) { return "retention-b200 0.1 (sm_100a)"; }
 
+int ret_device_error(void) {
+  const int a = ret::tc_state_device_error();
+  const int b = ret::tc_out_device_error();
+  if (a < 0 || b < 0) return -1;
+  return a ? a : b;
+}
+
 int ret_parallel(const void* q, const void* k, const void* v, const float* gammas, void* o,
                  int B, int H, int N, int dk, int dv, int dtype, float gn_eps, void* stream) {
   int s = check_seq_dims(B, H, N, dk, dv, dtype);
@@ -63,6 +81,11 @@ int ret_parallel(const void* q, const void* k, const void* v, const float* gamma
   if (!q || !k || !v || !o || !gammas) return RET_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == RET_BF16 && tc_dims(dk, dv)) {
+    if ((int64_t)((N + 127) / 128) > 65535) return RET_EUNSUPPORTED;
+    return cuda_status(ret::launch_tc_out(q, k, v, gammas, 0, nullptr, 0, o, B, H, N, dk, dv,
+                                          gn_eps, 1, st));
+  }
   return cuda_status(ret::launch_simt_parallel(q, k, v, gammas, o, B, H, N, dk, dv, dtype,
                                                gn_eps, st));
 }
@@ -70,6 +93,8 @@ int ret_parallel(const void* q, const void* k, const void* v, const float* gamma
 size_t ret_chunkwise_workspace(int B, int H, int N, int dk, int dv, int chunk, int dtype) {
   if (check_seq_dims(B, H, N, dk, dv, dtype) != RET_OK || chunk < 1) return 0;
   if (N == 0) return 0;
+  if (dtype == RET_BF16 && tc_dims(dk, dv) && tc_chunk(chunk))
+    return tc_workspace_bytes(B, H, N, dk, dv, chunk);
   return ret::simt_workspace_bytes(B, H, N, dk, dv, chunk);
 }
 
@@ -100,6 +125,21 @@ int ret_chunkwise(const void* q, const void* k, const void* v, const float* gamm
   const size_t need = ret_chunkwise_workspace(B, H, N, dk, dv, chunk, dtype);
   if (need > 0 && (!workspace || workspace_bytes < need)) return RET_EWORKSPACE;
   if (workspace && !aligned16(workspace)) return RET_EINVAL;
+  if (dtype == RET_BF16 && tc_dims(dk, dv) && tc_chunk(chunk)) {
+    const int nc = (N + chunk - 1) / chunk;
+    if ((int64_t)nc * (chunk / 128) > 65535) return RET_EUNSUPPORTED;
+    // The state kernel runs whenever a state enters, crosses a chunk boundary
+    // or is returned; it also stores the incoming state in workspace slot 0.
+    if (nc > 1 || state_out || state_in) {
+      int s2 = cuda_status(ret::launch_tc_state(k, v, gammas, chunk, state_in, state_out,
+                                                workspace, state_in != nullptr, B, H, N, dk, dv,
+                                                st));
+      if (s2) return s2;
+    }
+    return cuda_status(ret::launch_tc_out(q, k, v, gammas, chunk, workspace,
+                                          state_in != nullptr, o, B, H, N, dk, dv, gn_eps, 0,
+                                          st));
+  }
   return cuda_status(ret::launch_simt_chunkwise(q, k, v, gammas, chunk, state_in, state_out, o,
                                                 B, H, N, dk, dv, dtype, gn_eps, workspace, st));
 }

@@ -22,3 +22,17 @@ cudaError_t launch_simt_parallel(const void* q, const void* k, const void* v, co
                                  float eps, cudaStream_t st);
 
 }  // namespace ret
+
+namespace ret {
+
+// Tensor-core (tcgen05) kernels for bf16 inputs.
+cudaError_t launch_tc_state(const void* k, const void* v, const float* gammas, int chunk,
+                            const float* state_in, float* state_out, void* ws, int write_ws0,
+                            int B, int H, int N, int dk, int dv, cudaStream_t st);
+cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const float* gammas,
+                          int chunk, const void* ws, int has_state0, void* o, int B, int H, int N,
+                          int dk, int dv, float eps, int parallel_form, cudaStream_t st);
+int tc_state_device_error();
+int tc_out_device_error();
+
+}  // namespace ret

@@ -32,6 +32,13 @@ def ret(torch_cuda):
     return ret
 
 
+@pytest.fixture(autouse=True)
+def no_device_error(ret):
+    """Every test must end without a timed-out wait inside a kernel."""
+    yield
+    assert ret.device_error() == 0
+
+
 def _dev(t):
     return wl.to_torch(t, "cuda")
 
