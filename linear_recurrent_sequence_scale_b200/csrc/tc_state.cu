@@ -214,6 +214,8 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const int q = warp & 3;
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
     const int ncg = p.nt / 32;
+    // the first chunk's MMAs add onto gamma^L0 * state_in
+    const float g0 = gpow(lg, min(p.chunk, p.N));
     for (int hh = 0; hh < halves; ++hh) {
       const int r = 128 * hh + 32 * q + lane;
       for (int cgi = 0; cgi < ncg; ++cgi) {
@@ -232,6 +234,8 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
           }
           if (p.write_ws0)
             store_bf16_row32(p.ws + (((size_t)bh * p.nc) * p.dk + r) * p.dv + c, v);
+#pragma unroll
+          for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * g0);
         } else {
 #pragma unroll
           for (int x = 0; x < 32; ++x) v[x] = 0u;
