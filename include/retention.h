@@ -103,6 +103,32 @@ RET_API int ret_chunkwise(const void* q, const void* k, const void* v, const flo
                   int B, int H, int N, int dk, int dv, int dtype, float gn_eps,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* Bytes of device scratch compiled into the library for ret_chunkwise_noalloc. */
+#define RET_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * ret_chunkwise for callers that cannot allocate device memory: a plugin in
+ * a host runtime that owns every byte of device memory and offers it no
+ * allocator, or a latency-critical loop that must not call cudaMalloc/cudaFree
+ * (they can synchronise the device).  The paper has no counterpart; this is a
+ * deployment variant of the chunkwise form above, with the same arguments,
+ * results and errors except for the workspace.
+ *   - Scratch comes from a fixed device array of RET_NOALLOC_SCRATCH_BYTES
+ *     (64 MiB) inside the library, present on every GPU that loads it until the
+ *     process exits.  Sizes whose ret_chunkwise_workspace() exceeds it are
+ *     rejected with RET_EWORKSPACE before anything runs.
+ *   - The first call on each device looks the array's device address up (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call shares the one array: calls that overlap on the GPU race on
+ *     it and must be serialised by the caller.  Nothing in it needs to start
+ *     at zero; it keeps the last call's contents.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+RET_API int ret_chunkwise_noalloc(const void* q, const void* k, const void* v, const float* gammas,
+                          int chunk, const float* state_in, float* state_out, void* o,
+                          int B, int H, int N, int dk, int dv, int dtype, float gn_eps,
+                          void* stream);
+
 /*
  * One recurrent decode step for every (batch, head) pair ("RetNet - Retentive
  * Network - A Successor to Transformer for LLMs", Key Equations, Recurrent

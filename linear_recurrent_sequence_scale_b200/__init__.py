@@ -26,6 +26,8 @@ SIGNATURES = {
     "ret_parallel": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
     "ret_chunkwise_workspace": (_S, [_I, _I, _I, _I, _I, _I, _I]),
     "ret_chunkwise": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _S, _P]),
+    "ret_chunkwise_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F,
+                                   _P]),
     "ret_step": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "ret_status_string": (ctypes.c_char_p, [_I]),
     "ret_last_cuda_error": (_I, []),
