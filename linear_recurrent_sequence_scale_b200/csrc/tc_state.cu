@@ -1,26 +1,31 @@
-// Chunk-state scan on the tensor cores: bf16 operands, float32 state in TMEM.
+// Chunk-state scan on the tensor cores: bf16 operands, float32 state.
 //
 // "RetNet - Retentive Network - A Successor to Transformer for LLMs", Key
 // Equations, Chunkwise Recurrent: the state carried between chunks is
-//     R_i = gamma^L R_{i-1} + K_[i]^T (V_[i] (.) zeta),  zeta_j = gamma^(L-1-j)
+//     R_i = gamma^L R_{i-1} + H_i,   H_i = K_[i]^T (V_[i] (.) zeta),
+//     zeta_j = gamma^(L-1-j)
 // (the in-chunk decay zeta is the reading that makes the chunk state equal
 // the recurrent form summed over the chunk).
 //
-// One CTA owns one (batch, head) and NT (<= 128) state columns, all d_k rows
-// (two 128-row halves for d_k = 256), and walks the chunks in order:
-//   warp 0      TMA: K tile [T tokens][d_k] and V tile [T][NT] per stage
-//   warps 2-5   V (.) zeta, split into bf16 hi and lo parts when the final
-//               state is requested (hi + lo carries 16 mantissa bits, so the
-//               float32 state stays accurate to ~1e-6 instead of the 2^-9 of
-//               one bf16 rounding); hi is written in place of V
-//   warp 1      tcgen05.mma: R += K^T (V hi) [+ K^T (V lo)], M = 128 state
-//               rows, N = NT, K = 16 tokens, A and B both MN-major
-//   warps 6-9   at each chunk boundary: read R from TMEM, store it as bf16 to
-//               the workspace (the state entering the next chunk, read by the
-//               output kernel), scale it by gamma^L of the next chunk and
-//               write it back; after the last chunk store the float32 state.
-// Two CTAs fit on an SM (256 TMEM columns, ~97 KB shared memory each), so one
-// CTA's MMAs run while the other rescales its state.
+// One CTA owns one (batch, head), MH (1 or 2) 128-row halves of d_k and NT
+// (<= 128) state columns, and walks the chunks in order:
+//   warp 0      TMA: K tile [T tokens][128 MH d_k] and V tile [T][NT] per stage
+//   warps 2-5   V (.) zeta; when the final state is requested it is split
+//               into bf16 hi + lo parts (16 mantissa bits of the product
+//               reach the tensor core instead of 8), hi written in place of V
+//   warp 1      tcgen05.mma: H_i = K^T (V hi) [+ K^T (V lo)] into a TMEM
+//               accumulator that starts from zero in every chunk (M = 128
+//               state rows per half, N = NT, K = 16 tokens, MN-major operands)
+//   warps 6-13  the carried state R, float32 in a second TMEM region: at each
+//               chunk end they read H_i (then hand the accumulator back to the
+//               MMA warp), form gamma^L R + H_i with IEEE float32 FMAs, write
+//               R back, and store it as bf16 to the workspace (the state
+//               entering the next chunk, read by the output kernel) or, after
+//               the last chunk, as the float32 final state.
+// Accumulating each chunk afresh keeps the tensor core's running sums short
+// (one chunk), so the float32 state stays accurate over any sequence length.
+// MH = 2 halves the number of CTAs reading each K tile; MH = 1 gives twice
+// the CTAs for small batches.
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -32,40 +37,28 @@ namespace k2 {
 using namespace sm100;
 
 constexpr int T = 32;                  // tokens per stage
-constexpr int STAGES = 3;
+constexpr int NT = 128;                // state columns per CTA (d_v = 64 uses 64)
+constexpr int STAGES = 6;
 constexpr int BOX = T * 128;           // one [T][64] bf16 box: 4 KB
-constexpr int K_OFF = 0;               // 4 boxes (d_k up to 256)
-constexpr int V_OFF = 4 * BOX;         // 2 boxes (NT up to 128), becomes V hi
+constexpr int K_OFF = 0;               // 4 boxes: up to 256 rows of d_k
+constexpr int V_OFF = 4 * BOX;         // 2 boxes: NT columns of V, becomes V hi
 constexpr int LO_OFF = 6 * BOX;        // 2 boxes
 constexpr int STAGE_BYTES = 8 * BOX;   // 32 KB
 constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-constexpr int SMEM_BYTES = BAR_OFF + 256 + 1024;
-constexpr int THREADS = 320;
+constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;
+constexpr int THREADS = 448;           // 14 warps
 
 struct Params {
   const float* gammas;
   const float* state_in;
   float* state_out;
   __nv_bfloat16* ws;  // [B*H*nc][dk][dv]; slot i = state entering chunk i
-  int H, N, chunk, nc, dk, dv, nt;
+  int H, N, chunk, nc, dk, dv, nt, mh;
   int write_ws0;      // store state_in (as bf16) in slot 0
 };
 
-__device__ __forceinline__ void store_bf16_row32(__nv_bfloat16* dst, const uint32_t (&v)[32]) {
-  uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    uint4 w;
-    w.x = pack_bf16(__uint_as_float(v[8 * c + 0]), __uint_as_float(v[8 * c + 1]));
-    w.y = pack_bf16(__uint_as_float(v[8 * c + 2]), __uint_as_float(v[8 * c + 3]));
-    w.z = pack_bf16(__uint_as_float(v[8 * c + 4]), __uint_as_float(v[8 * c + 5]));
-    w.w = pack_bf16(__uint_as_float(v[8 * c + 6]), __uint_as_float(v[8 * c + 7]));
-    d[c] = w;
-  }
-}
-
 template <bool SPLIT>
-__global__ void __launch_bounds__(THREADS, 2)
+__global__ void __launch_bounds__(THREADS, 1)
 state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -75,20 +68,22 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
   uint64_t* full = bars;                 // TMA -> transform
   uint64_t* xf = bars + STAGES;          // transform -> MMA
   uint64_t* empty = bars + 2 * STAGES;   // MMA -> TMA
-  uint64_t* acc_ready = bars + 3 * STAGES;
-  uint64_t* acc_full = acc_ready + 1;
-  uint64_t* drain = acc_ready + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_ready + 3);
+  uint64_t* h_full = bars + 3 * STAGES;  // MMA -> epilogue
+  uint64_t* h_free = h_full + 1;         // epilogue -> MMA
+  uint64_t* drain = h_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(h_full + 3);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
+  const int bh = blockIdx.z;
   const int h = bh % p.H;
-  const int c0 = blockIdx.x * p.nt;
-  const int halves = (p.dk + 127) / 128;
-  const int kboxes = 2 * halves;  // d_k = 64 loads one out-of-range (zero) box as padding
+  const int r0 = blockIdx.y * 128 * p.mh;  // first d_k row of this CTA
+  const int c0 = blockIdx.x * p.nt;        // first state column
   const int vboxes = p.nt / 64;
-  const uint32_t tmem_cols = static_cast<uint32_t>(halves * p.nt);  // 64, 128 or 256
+  const int kboxes = 2 * p.mh;             // d_k = 64 loads an out-of-range (zero) box
+  // TMEM: H (accumulator) in [0, MH NT), R (carried state) in [MH NT, 2 MH NT)
+  const uint32_t rcol = static_cast<uint32_t>(p.mh * p.nt);
+  const uint32_t tmem_cols = 2 * rcol;     // 128, 256 or 512
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -96,8 +91,8 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       mbar_init(&xf[s], 4);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_ready, 4);
-    mbar_init(acc_full, 1);
+    mbar_init(h_full, 1);
+    mbar_init(h_free, 8);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -124,12 +119,11 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         const int L = min(p.chunk, p.N - cs);
         for (int j0 = 0; j0 < L; j0 += T, ++g) {
           const int slot = g % STAGES;
-          const uint32_t ph = (g / STAGES) & 1;
-          if (!mbar_wait(&empty[slot], ph ^ 1, 101)) { ok = false; break; }
+          if (!mbar_wait(&empty[slot], ((g / STAGES) & 1) ^ 1, 101)) { ok = false; break; }
           uint8_t* st = smem + slot * STAGE_BYTES;
           mbar_arrive_expect_tx(&full[slot], (kboxes + vboxes) * BOX);
           for (int b = 0; b < kboxes; ++b)
-            tma_load_3d(st + K_OFF + b * BOX, &tm_k, &full[slot], b * 64, cs + j0, bh);
+            tma_load_3d(st + K_OFF + b * BOX, &tm_k, &full[slot], r0 + b * 64, cs + j0, bh);
           for (int b = 0; b < vboxes; ++b)
             tma_load_3d(st + V_OFF + b * BOX, &tm_v, &full[slot], c0 + b * 64, cs + j0, bh);
         }
@@ -145,29 +139,32 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       int g = 0;
       bool ok = true;
       for (int ci = 0; ci < p.nc && ok; ++ci) {
-        if (!mbar_wait(acc_ready, ci & 1, 102)) { ok = false; break; }
+        // the epilogue must have read H_{ci-1} before it is overwritten
+        if (ci >= 1 && !mbar_wait(h_free, (ci - 1) & 1, 102)) { ok = false; break; }
         tc_fence_after();
         const int L = min(p.chunk, p.N - ci * p.chunk);
+        bool first = true;
         for (int j0 = 0; j0 < L; j0 += T, ++g) {
           const int slot = g % STAGES;
-          const uint32_t ph = (g / STAGES) & 1;
-          if (!mbar_wait(&xf[slot], ph, 103)) { ok = false; break; }
+          if (!mbar_wait(&xf[slot], (g / STAGES) & 1, 103)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sb = smem_u32(smem + slot * STAGE_BYTES);
 #pragma unroll
           for (int kk = 0; kk < T / 16; ++kk) {
             const uint64_t bhi = sdesc_sw128(sb + V_OFF + kk * 2048, BOX, 1024);
             const uint64_t blo = sdesc_sw128(sb + LO_OFF + kk * 2048, BOX, 1024);
-            for (int hh = 0; hh < halves; ++hh) {
+            for (int hh = 0; hh < p.mh; ++hh) {
               const uint64_t a = sdesc_sw128(sb + K_OFF + 2 * hh * BOX + kk * 2048, BOX, 1024);
-              umma_bf16_ss(tmem + hh * p.nt, a, bhi, idesc, 1u);
-              if (SPLIT) umma_bf16_ss(tmem + hh * p.nt, a, blo, idesc, 1u);
+              const uint32_t d = tmem + hh * p.nt;
+              umma_bf16_ss(d, a, bhi, idesc, first ? 0u : 1u);
+              if (SPLIT) umma_bf16_ss(d, a, blo, idesc, 1u);
             }
+            first = false;
           }
           umma_commit(&empty[slot]);
         }
         if (!ok) break;
-        umma_commit(acc_full);
+        umma_commit(h_full);
       }
       umma_commit(drain);
       mbar_wait(drain, 0, 109);
@@ -182,11 +179,10 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       const int L = min(p.chunk, p.N - ci * p.chunk);
       for (int j0 = 0; j0 < L; j0 += T, ++g) {
         const int slot = g % STAGES;
-        const uint32_t ph = (g / STAGES) & 1;
-        if (!mbar_wait(&full[slot], ph, 104)) { ok = false; break; }
+        if (!mbar_wait(&full[slot], (g / STAGES) & 1, 104)) { ok = false; break; }
         const uint32_t sb = smem_u32(smem + slot * STAGE_BYTES);
         for (int e = tt; e < nchunks; e += 128) {
-          const int box = e >> 8;           // 256 16-byte chunks per box
+          const int box = e >> 8;            // 256 16-byte chunks per box
           const int within = e & 255;
           const int j = j0 + (within >> 3);  // token row of this chunk
           const float z = (j < L) ? gpow(lg, L - 1 - j) : 0.f;
@@ -210,66 +206,88 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       }
     }
   } else {
-    // ---------------- state epilogue (TMEM lanes 32q..32q+31) ----------------
-    const int q = warp & 3;
+    // ---------------- carried state (float32, TMEM region R) ----------------
+    const int q = warp & 3;                   // TMEM lane quadrant
+    const int part = (warp - 6) >> 2;         // which half of the NT columns
+    const int ncol = p.nt / 2;                // 64 (or 32 when d_v = 64)
+    const int row = 32 * q + lane;            // state row within a d_k half
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-    const int ncg = p.nt / 32;
-    // the first chunk's MMAs add onto gamma^L0 * state_in
-    const float g0 = gpow(lg, min(p.chunk, p.N));
-    for (int hh = 0; hh < halves; ++hh) {
-      const int r = 128 * hh + 32 * q + lane;
-      for (int cgi = 0; cgi < ncg; ++cgi) {
+    const int cb = c0 + part * ncol;          // first global column of this thread
+    // R <- state_in (or zero); slot 0 of the workspace <- bf16(state_in)
+    for (int hh = 0; hh < p.mh; ++hh) {
+      const int r = r0 + 128 * hh + row;
+      const bool live = r < p.dk;
+      for (int x0 = 0; x0 < ncol; x0 += 32) {
         uint32_t v[32];
-        const int c = c0 + 32 * cgi;
-        if (p.state_in && r < p.dk) {
+        if (p.state_in && live) {
           const float4* src =
-              reinterpret_cast<const float4*>(p.state_in + ((size_t)bh * p.dk + r) * p.dv + c);
+              reinterpret_cast<const float4*>(p.state_in + ((size_t)bh * p.dk + r) * p.dv + cb + x0);
 #pragma unroll
           for (int x = 0; x < 8; ++x) {
             const float4 f = src[x];
-            v[4 * x + 0] = __float_as_uint(f.x);
+            v[4 * x] = __float_as_uint(f.x);
             v[4 * x + 1] = __float_as_uint(f.y);
             v[4 * x + 2] = __float_as_uint(f.z);
             v[4 * x + 3] = __float_as_uint(f.w);
           }
-          if (p.write_ws0)
-            store_bf16_row32(p.ws + (((size_t)bh * p.nc) * p.dk + r) * p.dv + c, v);
+          if (p.write_ws0) {
+            uint4* dst = reinterpret_cast<uint4*>(
+                p.ws + (((size_t)bh * p.nc) * p.dk + r) * p.dv + cb + x0);
 #pragma unroll
-          for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * g0);
+            for (int x = 0; x < 4; ++x)
+              dst[x] = make_uint4(
+                  pack_bf16(__uint_as_float(v[8 * x]), __uint_as_float(v[8 * x + 1])),
+                  pack_bf16(__uint_as_float(v[8 * x + 2]), __uint_as_float(v[8 * x + 3])),
+                  pack_bf16(__uint_as_float(v[8 * x + 4]), __uint_as_float(v[8 * x + 5])),
+                  pack_bf16(__uint_as_float(v[8 * x + 6]), __uint_as_float(v[8 * x + 7])));
+          }
         } else {
 #pragma unroll
           for (int x = 0; x < 32; ++x) v[x] = 0u;
         }
-        tmem_st32(tmem + lane_addr + hh * p.nt + 32 * cgi, v);
+        tmem_st32(tmem + lane_addr + rcol + hh * p.nt + part * ncol + x0, v);
       }
     }
     tmem_wait_st();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(acc_ready);
-
     for (int ci = 0; ci < p.nc; ++ci) {
-      if (!mbar_wait(acc_full, ci & 1, 105)) break;
+      if (!mbar_wait(h_full, ci & 1, 105)) break;
       tc_fence_after();
+      const float gL = gpow(lg, min(p.chunk, p.N - ci * p.chunk));
       const bool last = ci == p.nc - 1;
-      const float gnext = last ? 0.f : gpow(lg, min(p.chunk, p.N - (ci + 1) * p.chunk));
-      for (int hh = 0; hh < halves; ++hh) {
-        const int r = 128 * hh + 32 * q + lane;
-        for (int cgi = 0; cgi < ncg; ++cgi) {
-          const int c = c0 + 32 * cgi;
-          const uint32_t ta = tmem + lane_addr + hh * p.nt + 32 * cgi;
-          uint32_t v[32];
-          tmem_ld32(ta, v);
-          tmem_wait_ld();
-          if (!last) {
-            if (r < p.dk)
-              store_bf16_row32(p.ws + (((size_t)bh * p.nc + ci + 1) * p.dk + r) * p.dv + c, v);
+      // R <- gamma^L R + H, 32 columns at a time; the MMA warp reuses H for the
+      // next chunk only after every thread has read it (h_free).  This kernel
+      // is bound by its loads, not by the tensor core, so that wait is cheap.
 #pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * gnext);
-            tmem_st32(ta, v);
-          } else if (p.state_out && r < p.dk) {
-            float4* dst =
-                reinterpret_cast<float4*>(p.state_out + ((size_t)bh * p.dk + r) * p.dv + c);
+      for (int hh = 0; hh < 2; ++hh) {
+        if (hh >= p.mh) continue;
+        const int r = r0 + 128 * hh + row;
+        const bool live = r < p.dk;
+#pragma unroll
+        for (int x0 = 0; x0 < 64; x0 += 32) {
+          if (x0 >= ncol) continue;
+          const uint32_t hoff = lane_addr + hh * p.nt + part * ncol + x0;
+          uint32_t hv[32], v[32];
+          tmem_ld32(tmem + hoff, hv);
+          tmem_ld32(tmem + rcol + hoff, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            v[x] = __float_as_uint(fmaf(gL, __uint_as_float(v[x]), __uint_as_float(hv[x])));
+          if (!last) tmem_st32(tmem + rcol + hoff, v);
+          if (!live) continue;
+          if (!last) {
+            uint4* dst = reinterpret_cast<uint4*>(
+                p.ws + (((size_t)bh * p.nc + ci + 1) * p.dk + r) * p.dv + cb + x0);
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+              dst[x] = make_uint4(
+                  pack_bf16(__uint_as_float(v[8 * x]), __uint_as_float(v[8 * x + 1])),
+                  pack_bf16(__uint_as_float(v[8 * x + 2]), __uint_as_float(v[8 * x + 3])),
+                  pack_bf16(__uint_as_float(v[8 * x + 4]), __uint_as_float(v[8 * x + 5])),
+                  pack_bf16(__uint_as_float(v[8 * x + 6]), __uint_as_float(v[8 * x + 7])));
+          } else if (p.state_out) {
+            float4* dst = reinterpret_cast<float4*>(p.state_out + ((size_t)bh * p.dk + r) * p.dv +
+                                                    cb + x0);
 #pragma unroll
             for (int x = 0; x < 8; ++x)
               dst[x] = make_float4(__uint_as_float(v[4 * x]), __uint_as_float(v[4 * x + 1]),
@@ -277,12 +295,10 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
           }
         }
       }
-      if (!last) {
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acc_ready);
-      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(h_free);
     }
   }
 
@@ -319,9 +335,16 @@ cudaError_t launch_tc_state(const void* k, const void* v, const float* gammas, i
   p.nc = cdiv(N, chunk);
   p.dk = dk;
   p.dv = dv;
-  p.nt = dv < 128 ? dv : 128;
+  p.nt = dv < NT ? dv : NT;
   p.write_ws0 = write_ws0;
-  dim3 grid(dv / p.nt, (unsigned)BH);
+  // Both d_k halves in one CTA (K read by half as many CTAs) when that still
+  // gives at least one CTA per SM; otherwise one half per CTA.
+  int dev = 0, nsm = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int halves = cdiv(dk, 128);
+  p.mh = (halves == 2 && BH * (uint64_t)(dv / p.nt) >= (uint64_t)nsm) ? 2 : 1;
+  dim3 grid(dv / p.nt, halves / p.mh, (unsigned)BH);
   if (state_out) {
     auto fn = state_scan_tc<true>;
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
