@@ -26,6 +26,8 @@
 // column down, multiplying by gamma per column, one exp2 per 32 columns.
 // S_t's buffer is rewritten by Q K_{t+2}^T only after the MMA reading P_t was
 // issued; tcgen05.mma from one thread executes in issue order.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -86,6 +88,22 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
 }
 
 // Chan et al.: merge (n_b, mean_b, m2_b) into (n_a, mean_a, m2_a).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, uint32_t src, int x, int y,
+                                             int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
 __device__ __forceinline__ void chan_merge(float& n_a, float& mean_a, float& m2_a, float n_b,
                                            float mean_b, float m2_b) {
   const float n = n_a + n_b;
@@ -95,11 +113,11 @@ __device__ __forceinline__ void chan_merge(float& n_a, float& mean_a, float& m2_
   n_a = n;
 }
 
-template <bool GN, int NQB>
+template <bool GN, int NQB, int KQ>
 __global__ void __launch_bounds__(THREADS, 1)
 chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_r,
-             const Params p) {
+             const __grid_constant__ CUtensorMap tm_o, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uintptr_t raw = reinterpret_cast<uintptr_t>(smem_raw);
   const uintptr_t aligned = (raw + 1023) & ~static_cast<uintptr_t>(1023);
@@ -112,8 +130,9 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   constexpr int RING_OFF = Layout<NQB>::RING_OFF;
   const int slice = blockIdx.x;
   const int c0 = slice * p.dvs;
-  const int kq = p.dk / 64;           // 64-wide blocks of d_k
-  const int kst = (kq + 1) / 2;       // K-tile stages (two blocks each)
+  constexpr int kq = KQ;              // 64-wide blocks of d_k
+  constexpr int kst = (KQ + 1) / 2;   // K-tile stages (two blocks each)
+  constexpr int KST = kst;
   const int vb = p.dvs / 64;          // 64-wide blocks of the column slice
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
@@ -141,7 +160,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&q_full[b], 1);
-      mbar_init(&q_empty[b], 1);
+      mbar_init(&q_empty[b], 1);  // arrived by the epilogue: the buffer also stages O
       mbar_init(&s_full[b], 1);
       mbar_init(&p_full[b], 4);
       mbar_init(&gn_bar[b], 128);
@@ -261,10 +280,13 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         umma_commit(&empty[g % RING]);
         ++g;
       };
+      // Descriptors: one full descriptor per operand buffer, then constant
+      // offsets (the start address sits in the low bits, in 16-byte units), so
+      // the issuing thread spends its time on MMAs, not on address arithmetic.
       for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++k) {
         const Tile x = decode_tile(p, tile);
         const int qb = k % NQB;
-        const uint32_t q_addr = smem_u32(smem + Q_OFF + qb * QBUF);
+        const uint64_t qd = sdesc_sw128(smem_u32(smem + Q_OFF + qb * QBUF), 16, 1024);
         if (!mbar_wait(&q_full[qb], (k / NQB) & 1, 204)) { ok = false; break; }
         tc_fence_after();
         const int s0 = sc;  // S-buffer use index of this tile's key tile 0
@@ -272,18 +294,20 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           if (t < x.nt) {
             const int b = sc & 1;
             const uint32_t d = tmem + b * BN;
-            for (int s = 0; s < kst && ok; ++s) {
-              uint32_t sa;
-              if (!take(sa)) { ok = false; break; }
-              const int nb = min(2, kq - 2 * s);
-              for (int bb = 0; bb < nb; ++bb)
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                  const int kb = 2 * s + bb;
-                  const uint64_t a = sdesc_sw128(q_addr + kb * QBOX + kk * 32, 16, 1024);
-                  const uint64_t bd = sdesc_sw128(sa + bb * QBOX + kk * 32, 16, 1024);
-                  umma_bf16_ss(d, a, bd, id_qk, (kb | kk) ? 1u : 0u);
-                }
+            for (int s = 0; s < KST; ++s) {
+              uint32_t sa;
+              if (!ok || !take(sa)) { ok = false; break; }
+              const uint64_t kd = sdesc_sw128(sa, 16, 1024);
+#pragma unroll
+              for (int bb = 0; bb < 2; ++bb) {
+                if (2 * s + bb >= KQ) break;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  umma_bf16_ss(d, qd + (((2 * s + bb) * QBOX + kk * 32) >> 4),
+                               kd + ((bb * QBOX + kk * 32) >> 4), id_qk,
+                               (s | bb | kk) ? 1u : 0u);
+              }
               give();
             }
             if (!ok) break;
@@ -298,15 +322,16 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             if (tp == 0 && k >= 1 && !mbar_wait(o_free, (k - 1) & 1, 206)) { ok = false; break; }
             tc_fence_after();
             const uint32_t pa = tmem + b * BN;  // P_t: 64 columns of packed bf16
-            for (int s = 0; s < 2 && ok; ++s) {
-              uint32_t sa;
-              if (!take(sa)) { ok = false; break; }
+            const uint32_t acc0 = tp ? 1u : 0u;
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const int key = 64 * s + 16 * kk;
-                const uint64_t bd = sdesc_sw128(sa + kk * 2048, VBOX, 1024);
-                umma_bf16_ts(o_tm, pa + key / 2, bd, id_pv, (tp | s | kk) ? 1u : 0u);
-              }
+            for (int s = 0; s < 2; ++s) {
+              uint32_t sa;
+              if (!ok || !take(sa)) { ok = false; break; }
+              const uint64_t vd = sdesc_sw128(sa, VBOX, 1024);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16_ts(o_tm, pa + 32 * s + 8 * kk, vd + ((kk * 2048) >> 4), id_pv,
+                             (s | kk) ? 1u : acc0);
               give();
             }
           }
@@ -315,19 +340,18 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (!mbar_wait(qt_full, k & 1, 207)) { ok = false; break; }
         tc_fence_after();
         if (x.has_r) {
-          for (int s = 0; s < kq && ok; ++s) {
-            uint32_t sa;
-            if (!take(sa)) { ok = false; break; }
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t a = sdesc_sw128(q_addr + s * QBOX + kk * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(sa + kk * 2048, VBOX, 1024);
-              umma_bf16_ss(o_tm, a, bd, id_pv, 1u);
-            }
+          for (int s = 0; s < KQ; ++s) {
+            uint32_t sa;
+            if (!ok || !take(sa)) { ok = false; break; }
+            const uint64_t rd = sdesc_sw128(sa, VBOX, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_ss(o_tm, qd + ((s * QBOX + kk * 32) >> 4), rd + ((kk * 2048) >> 4), id_pv,
+                           1u);
             give();
           }
         }
-        umma_commit(&q_empty[qb]);
         umma_commit(o_full);
       }
       umma_commit(drain);
@@ -453,9 +477,11 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         mean = m_a;
         inv = 1.0f / sqrtf(q_a / static_cast<float>(p.dv) + p.eps);
       }
-      const int n = x.n0 + i;
-      const bool live = n < p.N && n < x.cs + p.chunk;
-      __nv_bfloat16* orow = p.o + ((size_t)x.bh * p.N + (live ? n : 0)) * p.dv + c0;
+      // Stage bf16 O in this tile's Q buffer (its last reader, the inter-chunk
+      // MMA, is done) as [64-column block][128 rows][128 B] with the 128-byte
+      // swizzle, then write it with coalesced TMA stores; rows past N are
+      // clipped by the tensor map.
+      const uint32_t stage_a = smem_u32(smem + Q_OFF + (k % NQB) * QBUF) + i * 128;
       for (int cg = 0; cg < ncg; ++cg) {
         uint32_t v[32];
         tmem_ld32(o_tm + 32 * cg, v);
@@ -465,18 +491,27 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           __syncwarp();
           if (lane == 0) mbar_arrive(o_free);  // O may be overwritten now
         }
-        if (live) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cg);
+        uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t w4[4];
+        for (int xx = 0; xx < 16; ++xx)
+          pk[xx] = pack_bf16((__uint_as_float(v[2 * xx]) - mean) * inv,
+                             (__uint_as_float(v[2 * xx + 1]) - mean) * inv);
+        const uint32_t rowa = stage_a + (cg >> 1) * QBOX;
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w4[e] = pack_bf16((__uint_as_float(v[8 * c + 2 * e]) - mean) * inv,
-                                (__uint_as_float(v[8 * c + 2 * e + 1]) - mean) * inv);
-            dst[c] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
+        for (int c = 0; c < 4; ++c) {
+          const int phys = (((cg & 1) * 4 + c) ^ (i & 7));
+          st_shared_v4(rowa + phys * 16, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         }
+      }
+      fence_proxy_async_smem();
+      epi_bar();
+      if (warp == 6 && lane == 0) {
+        const uint32_t sb = smem_u32(smem + Q_OFF + (k % NQB) * QBUF);
+        for (int b = 0; b < p.dvs / 64; ++b)
+          tma_store_3d(&tm_o, sb + b * QBOX, c0 + b * 64, x.n0, x.bh);
+        bulk_commit();
+        bulk_wait_read0();
+        mbar_arrive(&q_empty[k % NQB]);  // the loader may refill the buffer
       }
     }
   }
@@ -527,9 +562,10 @@ cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const flo
   if (nclusters > p.ntiles) nclusters = p.ntiles;
   if (nclusters < 1) nclusters = 1;
 
-  CUtensorMap tm_q, tm_k, tm_v, tm_r;
+  CUtensorMap tm_q, tm_k, tm_v, tm_r, tm_o;
   if ((e = make_tmap_bf16_3d(&tm_q, q, dk, N, BH, 64, BM)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_3d(&tm_k, k, dk, N, BH, 64, BN)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_3d(&tm_o, o, dv, N, BH, 64, BM)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_3d(&tm_v, v, dv, N, BH, 64, 64)) != cudaSuccess) return e;
   if (ws) {
     if ((e = make_tmap_bf16_3d(&tm_r, ws, dv, dk, BH * p.nc, 64, 64)) != cudaSuccess) return e;
@@ -550,17 +586,38 @@ cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const flo
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   // Short tiles (chunkwise) gain most from loading the next Q early; long
-  // tiles (parallel form) from a deeper ring.
+  // tiles (parallel form) from a deeper ring (both measured on B200).
   const int nqb = parallel_form ? 1 : 2;
+  // A persistent grid must not exceed the clusters that can be resident at
+  // once: clusters live inside one GPC, and GPCs do not split evenly into
+  // clusters of 2 or 4, so SM count / cluster size can overshoot.
   auto launch = [&](auto fn) -> cudaError_t {
     cudaError_t e2 = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           SMEM_BYTES);
     if (e2 != cudaSuccess) return e2;
-    return cudaLaunchKernelEx(&cfg, fn, tm_q, tm_k, tm_v, tm_r, p);
+    if (cfg.gridDim.x > 1) {
+      e2 = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+      if (e2 != cudaSuccess) return e2;
+      int max_clusters = 0;
+      e2 = cudaOccupancyMaxActiveClusters(&max_clusters, fn, &cfg);
+      if (e2 != cudaSuccess) return e2;
+      if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+      if (cfg.gridDim.y > static_cast<unsigned>(max_clusters)) cfg.gridDim.y = max_clusters;
+    }
+    return cudaLaunchKernelEx(&cfg, fn, tm_q, tm_k, tm_v, tm_r, tm_o, p);
   };
+  auto by_dk = [&](auto gn, auto q) -> cudaError_t {
+    constexpr bool G = decltype(gn)::value;
+    constexpr int QB = decltype(q)::value;
+    if (dk == 64) return launch(chunk_out_tc<G, QB, 1>);
+    if (dk == 128) return launch(chunk_out_tc<G, QB, 2>);
+    return launch(chunk_out_tc<G, QB, 4>);
+  };
+  using T1 = std::integral_constant<int, 1>;
+  using T2 = std::integral_constant<int, 2>;
   if (eps >= 0.f)
-    return nqb == 1 ? launch(chunk_out_tc<true, 1>) : launch(chunk_out_tc<true, 2>);
-  return nqb == 1 ? launch(chunk_out_tc<false, 1>) : launch(chunk_out_tc<false, 2>);
+    return nqb == 1 ? by_dk(std::true_type{}, T1{}) : by_dk(std::true_type{}, T2{});
+  return nqb == 1 ? by_dk(std::false_type{}, T1{}) : by_dk(std::false_type{}, T2{});
 }
 
 }  // namespace ret
