@@ -68,9 +68,8 @@ const char* ret_version(void) { return "retention-b200 0.1 (sm_100a)"; }
 int ret_device_error(void) {
   const int a = ret::tc_state_device_error();
   const int b = ret::tc_out_device_error();
-  const int c = ret::tc_out2_device_error();
-  if (a < 0 || b < 0 || c < 0) return -1;
-  return a ? a : (b ? b : c);
+  if (a < 0 || b < 0) return -1;
+  return a ? a : b;
 }
 
 int ret_parallel(const void* q, const void* k, const void* v, const float* gammas, void* o,
@@ -84,9 +83,6 @@ int ret_parallel(const void* q, const void* k, const void* v, const float* gamma
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == RET_BF16 && tc_dims(dk, dv)) {
     if ((int64_t)((N + 127) / 128) > 65535) return RET_EUNSUPPORTED;
-    if (ret::tc_out2_supported(dk, dv, 0, 1))
-      return cuda_status(ret::launch_tc_out2(q, k, v, gammas, 0, nullptr, 0, o, B, H, N, dk, dv,
-                                             gn_eps, 1, st));
     return cuda_status(ret::launch_tc_out(q, k, v, gammas, 0, nullptr, 0, o, B, H, N, dk, dv,
                                           gn_eps, 1, st));
   }
@@ -140,10 +136,6 @@ int ret_chunkwise(const void* q, const void* k, const void* v, const float* gamm
                                                 st));
       if (s2) return s2;
     }
-    if (ret::tc_out2_supported(dk, dv, chunk, 0))
-      return cuda_status(ret::launch_tc_out2(q, k, v, gammas, chunk, workspace,
-                                             state_in != nullptr, o, B, H, N, dk, dv, gn_eps, 0,
-                                             st));
     return cuda_status(ret::launch_tc_out(q, k, v, gammas, chunk, workspace,
                                           state_in != nullptr, o, B, H, N, dk, dv, gn_eps, 0,
                                           st));

@@ -32,12 +32,7 @@ cudaError_t launch_tc_state(const void* k, const void* v, const float* gammas, i
 cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const float* gammas,
                           int chunk, const void* ws, int has_state0, void* o, int B, int H, int N,
                           int dk, int dv, float eps, int parallel_form, cudaStream_t st);
-cudaError_t launch_tc_out2(const void* q, const void* k, const void* v, const float* gammas,
-                           int chunk, const void* ws, int has_state0, void* o, int B, int H, int N,
-                           int dk, int dv, float eps, int parallel_form, cudaStream_t st);
-bool tc_out2_supported(int dk, int dv, int chunk, int parallel_form);
 int tc_state_device_error();
 int tc_out_device_error();
-int tc_out2_device_error();
 
 }  // namespace ret

@@ -10,13 +10,13 @@
 // One CTA owns one (batch, head), MH (1 or 2) 128-row halves of d_k and NT
 // (<= 128) state columns, and walks the chunks in order:
 //   warp 0      TMA: K tile [T tokens][128 MH d_k] and V tile [T][NT] per stage
-//   warps 2-5   V (.) zeta; when the final state is requested it is split
+//   warps 2-9   V (.) zeta; when the final state is requested it is split
 //               into bf16 hi + lo parts (16 mantissa bits of the product
 //               reach the tensor core instead of 8), hi written in place of V
 //   warp 1      tcgen05.mma: H_i = K^T (V hi) [+ K^T (V lo)] into a TMEM
 //               accumulator that starts from zero in every chunk (M = 128
 //               state rows per half, N = NT, K = 16 tokens, MN-major operands)
-//   warps 6-13  the carried state R, float32 in a second TMEM region: at each
+//   warps 10-17 the carried state R, float32 in a second TMEM region: at each
 //               chunk end they read H_i (then hand the accumulator back to the
 //               MMA warp), form gamma^L R + H_i with IEEE float32 FMAs, write
 //               R back, and store it as bf16 to the workspace (the state
@@ -46,7 +46,9 @@ constexpr int LO_OFF = 6 * BOX;        // 2 boxes
 constexpr int STAGE_BYTES = 8 * BOX;   // 32 KB
 constexpr int BAR_OFF = STAGES * STAGE_BYTES;
 constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;
-constexpr int THREADS = 448;           // 14 warps
+constexpr int XF_WARPS = 8;            // V (.) zeta warps
+constexpr int EPI_WARP0 = 2 + XF_WARPS;  // first state warp
+constexpr int THREADS = (EPI_WARP0 + 8) * 32;  // 18 warps
 
 struct Params {
   const float* gammas;
@@ -88,7 +90,7 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&xf[s], 4);
+      mbar_init(&xf[s], XF_WARPS);
       mbar_init(&empty[s], 1);
     }
     mbar_init(h_full, 1);
@@ -169,10 +171,17 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       umma_commit(drain);
       mbar_wait(drain, 0, 109);
     }
-  } else if (warp < 6) {
+  } else if (warp < EPI_WARP0) {
     // ---------------- V (.) zeta, hi/lo split ----------------
+    // A stage holds T token rows of NT columns (16-byte chunks, 8 per 64-column
+    // box row).  Each thread owns consecutive chunks of one token row, so it
+    // needs one zeta per stage and can issue all its loads before any store.
     const int tt = threadIdx.x - 64;
-    const int nchunks = vboxes * (BOX / 16);
+    constexpr int NXT = XF_WARPS * 32;
+    const int cpr = p.nt / 8;                  // 16-byte chunks per token row
+    const int per = (T * cpr) / NXT;           // chunks per thread: 2 (NT = 128) or 1
+    const int row = (tt * per) / cpr;
+    const int c_first = (tt * per) % cpr;
     int g = 0;
     bool ok = true;
     for (int ci = 0; ci < p.nc && ok; ++ci) {
@@ -181,24 +190,33 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         const int slot = g % STAGES;
         if (!mbar_wait(&full[slot], (g / STAGES) & 1, 104)) { ok = false; break; }
         const uint32_t sb = smem_u32(smem + slot * STAGE_BYTES);
-        for (int e = tt; e < nchunks; e += 128) {
-          const int box = e >> 8;            // 256 16-byte chunks per box
-          const int within = e & 255;
-          const int j = j0 + (within >> 3);  // token row of this chunk
-          const float z = (j < L) ? gpow(lg, L - 1 - j) : 0.f;
-          const uint32_t off = box * BOX + within * 16;
-          const uint4 v = ld_shared_v4(sb + V_OFF + off);
-          const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-          uint32_t hi[4], lo[4];
+        const int j = j0 + row;
+        const float z = (j < L) ? gpow(lg, L - 1 - j) : 0.f;
+        uint32_t off[2];
+        uint4 v[2];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const float a = bf16lo_to_f32(in[c]) * z;
-            const float b = bf16hi_to_f32(in[c]) * z;
-            hi[c] = pack_bf16(a, b);
-            if (SPLIT) lo[c] = pack_bf16(a - bf16lo_to_f32(hi[c]), b - bf16hi_to_f32(hi[c]));
+        for (int u = 0; u < 2; ++u) {
+          if (u < per) {
+            const int c = c_first + u;         // chunk within the row: box c/8, chunk c%8
+            off[u] = (c >> 3) * BOX + row * 128 + (c & 7) * 16;
+            v[u] = ld_shared_v4(sb + V_OFF + off[u]);
           }
-          st_shared_v4(sb + V_OFF + off, hi[0], hi[1], hi[2], hi[3]);
-          if (SPLIT) st_shared_v4(sb + LO_OFF + off, lo[0], lo[1], lo[2], lo[3]);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (u < per) {
+            const uint32_t in[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const float a = bf16lo_to_f32(in[c]) * z;
+              const float b = bf16hi_to_f32(in[c]) * z;
+              hi[c] = pack_bf16(a, b);
+              if (SPLIT) lo[c] = pack_bf16(a - bf16lo_to_f32(hi[c]), b - bf16hi_to_f32(hi[c]));
+            }
+            st_shared_v4(sb + V_OFF + off[u], hi[0], hi[1], hi[2], hi[3]);
+            if (SPLIT) st_shared_v4(sb + LO_OFF + off[u], lo[0], lo[1], lo[2], lo[3]);
+          }
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -208,7 +226,7 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
   } else {
     // ---------------- carried state (float32, TMEM region R) ----------------
     const int q = warp & 3;                   // TMEM lane quadrant
-    const int part = (warp - 6) >> 2;         // which half of the NT columns
+    const int part = (warp - EPI_WARP0) >> 2;  // which half of the NT columns
     const int ncol = p.nt / 2;                // 64 (or 32 when d_v = 64)
     const int row = 32 * q + lane;            // state row within a d_k half
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
