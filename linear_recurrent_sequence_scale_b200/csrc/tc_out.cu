@@ -192,17 +192,32 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       if (p.chunked) tma_prefetch_desc(&tm_r);
       int g = 0, k = 0;
       bool ok = true;
-      auto load_q = [&](int kk, const Tile& x) -> bool {
-        const int qb = kk % NQB;
-        if (!mbar_wait(&q_empty[qb], ((kk / NQB) & 1) ^ 1, 201)) return false;
+      // Q of this CTA's tile sequence number qn goes to buffer qn % NQB once
+      // that buffer is free (the epilogue of tile qn - NQB has stored its O
+      // from it).  The loader never blocks on that while it still has ring
+      // stages to issue: it polls between stages and waits only when the tile
+      // that needs the Q starts.
+      int qn = 0;  // next Q to load (tile sequence number)
+      auto issue_q = [&](bool block) -> bool {
+        const int tile = tile0 + qn * tstep;
+        if (tile >= p.ntiles || qn > k + (NQB - 1)) return true;
+        const int qb = qn % NQB;
+        const uint32_t par = ((qn / NQB) & 1) ^ 1;
+        if (block) {
+          if (!mbar_wait(&q_empty[qb], par, 201)) return false;
+        } else if (!mbar_try_wait(&q_empty[qb], par)) {
+          return true;
+        }
+        const Tile y = decode_tile(p, tile);
         mbar_arrive_expect_tx(&q_full[qb], kq * QBOX);
         for (int b = 0; b < kq; ++b)
-          tma_load_3d(smem + Q_OFF + qb * QBUF + b * QBOX, &tm_q, &q_full[qb], b * 64, x.n0,
-                      x.bh);
+          tma_load_3d(smem + Q_OFF + qb * QBUF + b * QBOX, &tm_q, &q_full[qb], b * 64, y.n0, y.bh);
+        ++qn;
         return true;
       };
       auto acquire = [&](uint32_t bytes, uint64_t*& bar) -> uint8_t* {
         const int slot = g % RING;
+        if (!issue_q(false)) return nullptr;
         if (!mbar_wait(&empty[slot], ((g / RING) & 1) ^ 1, 202)) return nullptr;
         bar = &full[slot];
         mbar_arrive_expect_tx(bar, bytes);
@@ -210,8 +225,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       };
       for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++k) {
         const Tile x = decode_tile(p, tile);
-        if (k == 0) ok = load_q(0, x);
-        bool next_q_done = false;
+        while (ok && qn <= k) ok = issue_q(true);  // this tile's own Q
         for (int t = 0; t <= x.nt && ok; ++t) {
           if (t < x.nt) {
             const int key0 = x.cs + t * BN;
@@ -222,17 +236,6 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
               if (!st) { ok = false; break; }
               for (int b = 0; b < nb; ++b)
                 tma_load_3d(st + b * QBOX, &tm_k, bar, (2 * s + b) * 64, key0, x.bh);
-            }
-          }
-          // Q loads once this tile's first K tile is queued: with two buffers
-          // the next tile's Q (its buffer was freed by the previous tile);
-          // with one buffer this tile's own Q, after the previous tile is done
-          if (!next_q_done && ok) {
-            next_q_done = true;
-            if (NQB == 2) {
-              if (tile + tstep < p.ntiles) ok = load_q(k + 1, decode_tile(p, tile + tstep));
-            } else if (k >= 1) {
-              ok = load_q(k, x);
             }
           }
           if (t >= 1 && ok) {
