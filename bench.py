@@ -10,7 +10,10 @@ d_v 512, chunk 512, bf16 inputs, decays gamma_h = 1 - 2^(-5-h).  The headline
 with CUDA events on the launching stream with the inputs resident in HBM.
 The inputs (3.2 GB per step) are far larger than the 126 MB L2, so no flush
 is needed between steps.  The same line carries:
-  roofline      the chunkwise call against the measured bf16 tensor peak
+  roofline      the chunk-output kernel (the larger of the two the chunkwise
+                call launches), timed live between events, against the
+                measured bf16 tensor peak; the state-scan kernel and the
+                whole call are reported beside it
   e2e           the same metric through the public API with pinned host
                 buffers: host->device copy of q, k, v and device->host copy
                 of o inside the timed region
@@ -63,6 +66,14 @@ def chunkwise_flops(B, H, N, dk, dv, C, state_in=False, state_out=False):
     inter = sum(2 * dk * dv * L for i, L in enumerate(Ls) if i > 0 or state_in)
     state = sum(2 * dk * dv * L for i, L in enumerate(Ls) if i < len(Ls) - 1 or state_out)
     return B * H * (intra + inter + state)
+
+
+def chunkwise_phase_flops(B, H, N, dk, dv, C, state_in=False, state_out=False):
+    """(states phase, output phase) shares of chunkwise_flops: the chunk
+    states K^T (V (.) zeta), and the intra-chunk plus cross-chunk outputs."""
+    Ls = chunk_lengths(N, C)
+    state = sum(2 * dk * dv * L for i, L in enumerate(Ls) if i < len(Ls) - 1 or state_out)
+    return B * H * state, chunkwise_flops(B, H, N, dk, dv, C, state_in, state_out) - B * H * state
 
 
 def chunkwise_bytes(B, H, N, dk, dv, elem=2, state_in=False, state_out=False):
@@ -130,21 +141,26 @@ def global_throughput(units_per_rank_per_step: float, steps: int, world: int, t_
 # measurement helpers
 # ---------------------------------------------------------------------------
 
-def kernel_source_hash():
-    """Hash of the CUDA sources: stored profiler counters are only valid for it."""
+# Sources that decide what the chunk-output kernel does (its code, the
+# headers it includes and the tensor maps it is launched with).
+OUT_KERNEL_SOURCES = ("tc_out.cu", "sm100.cuh", "common.cuh", "kernels.h", "tmap.cu", "tmap.h")
+
+
+def kernel_source_hash(names=OUT_KERNEL_SOURCES):
+    """Hash of the CUDA sources of the chunk-output kernel: stored profiler
+    counters are only valid for it."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_recurrent_sequence_scale_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+    for name in sorted(names):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def stored_traffic(workload):
-    """DRAM bytes per call from the committed ncu summary, or None when the
-    kernels changed since it was taken."""
+    """DRAM bytes per launch of the chunk-output kernel from the committed ncu
+    summary, or None when that kernel changed since the capture."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -152,7 +168,7 @@ def stored_traffic(workload):
         d = json.load(f)
     if d.get("source_hash") != kernel_source_hash():
         return None
-    return d.get("per_call_bytes", {}).get(workload)
+    return d.get("per_launch_bytes", {}).get(workload)
 
 
 def load_peaks():
@@ -232,26 +248,37 @@ class ClockSampler:
                 "samples": len(loaded)}
 
 
-def timed(fn, steps, warmup, stream, device):
+def timed(fn, steps, warmup, stream, device, phases=None):
     """Run fn warmup times, then time exactly `steps` calls with CUDA events on
     `stream`, bracketed by a barrier and a device synchronize on both sides.
-    Returns (seconds of this rank, max seconds over ranks)."""
+    Returns (seconds of this rank, max seconds over ranks).  With `phases` (a
+    list of callables that together make one call of fn) each step runs the
+    phases with an event between them, and a third value lists the seconds
+    each phase took over all steps."""
     import torch
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize(device)
     barrier(device)
     torch.cuda.synchronize(device)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    nb = steps * (len(phases) if phases else 1) + 1
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(nb)]
+    j = 0
+    ev[0].record(stream)
     for _ in range(steps):
-        fn()
-    e1.record(stream)
+        for f in (phases or [fn]):
+            f()
+            j += 1
+            ev[j].record(stream)
     torch.cuda.synchronize(device)
     barrier(device)
-    t = e0.elapsed_time(e1) / 1e3
-    return t, max_over_ranks(t, device)
+    t = ev[0].elapsed_time(ev[-1]) / 1e3
+    if not phases:
+        return t, max_over_ranks(t, device)
+    P = len(phases)
+    per = [sum(ev[s * P + i].elapsed_time(ev[s * P + i + 1]) for s in range(steps)) / 1e3
+           for i in range(P)]
+    return t, max_over_ranks(t, device), per
 
 
 def make_qkv(torch, B, H, N, dk, dv, device, seed):
@@ -370,27 +397,43 @@ def run_ours(args):
     ws = torch.empty(ret.chunkwise_workspace_bytes(B, H, N, dk, dv, C, torch.bfloat16),
                      dtype=torch.uint8, device=device)
     step = lambda: ret.chunkwise(q, k, v, gam, C, gn_eps=eps, out=o, workspace=ws)
+    # the same call in its two phases, so that each kernel's time is measured
+    # live: ret_chunkwise is exactly these two calls on one stream
+    phases = [lambda: ret.chunkwise_states(k, v, gam, C, ws),
+              lambda: ret.chunkwise_output(q, k, v, gam, C, ws, gn_eps=eps, out=o)]
     clocks = ClockSampler(smi_index(local))
     clocks.start()
-    t_local, t_max = timed(step, args.steps, args.warmup, stream, device)
+    t_local, t_max, t_phase = timed(step, args.steps, args.warmup, stream, device, phases)
     clocks.stop()
     launches += 2 * args.steps  # state scan + chunk output per call
     tokens = B * N
     value = global_throughput(tokens, args.steps, world, t_max)
     F = chunkwise_flops(B, H, N, dk, dv, C)
+    F_states, F_out = chunkwise_phase_flops(B, H, N, dk, dv, C)
     Bytes = chunkwise_bytes(B, H, N, dk, dv)
     call_s = t_local / args.steps
-    achieved = F / call_s / 1e12
+    out_s = t_phase[1] / args.steps
+    states_s = t_phase[0] / args.steps
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    achieved = F_out / out_s / 1e12
     traffic = stored_traffic(WORKLOAD)
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,
-                "kernel": "ret_chunkwise (state scan + chunk output)",
+                "kernel": "chunk_out_tc (ret_chunkwise_output), the dominant kernel",
                 "peak_source": f"{peak_src} bf16 burst; sustained "
                                f"{peaks.get('bf16_tflops_sustained')}",
-                "algorithmic_flop_per_call": F, "algorithmic_bytes_per_call": Bytes,
-                "hbm_gbs_achieved": Bytes / call_s / 1e9,
-                "hbm_frac": Bytes / call_s / 1e9 / peaks.get("hbm_gbs", 6650.0)}
+                "algorithmic_flop_per_launch": F_out,
+                "kernel_ms": out_s * 1e3,
+                "share_of_step": out_s / call_s,
+                "other_kernel": {"name": "state_scan_tc (ret_chunkwise_states)",
+                                 "ms": states_s * 1e3, "algorithmic_flop": F_states,
+                                 "tflops": F_states / states_s / 1e12,
+                                 "frac": F_states / states_s / 1e12 / peak},
+                "whole_call": {"algorithmic_flop": F, "tflops": F / call_s / 1e12,
+                               "frac": F / call_s / 1e12 / peak,
+                               "algorithmic_bytes": Bytes,
+                               "hbm_gbs": Bytes / call_s / 1e9,
+                               "hbm_frac": Bytes / call_s / 1e9 / peaks.get("hbm_gbs", 6650.0)}}
     del ws
 
     # ---------------- e2e through the public API with host buffers ----------------

@@ -103,6 +103,38 @@ RET_API int ret_chunkwise(const void* q, const void* k, const void* v, const flo
                   int B, int H, int N, int dk, int dv, int dtype, float gn_eps,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * The chunkwise form in its two phases; ret_chunkwise is exactly
+ * ret_chunkwise_states followed by ret_chunkwise_output on one stream.
+ * ("RetNet - Retentive Network - A Successor to Transformer for LLMs", Key
+ * Equations, Chunkwise Recurrent: the states R_i form one pass, the outputs
+ * of all chunks the other.)  Callers use them to time the phases apart or to
+ * keep the chunk states of a prefill.
+ *
+ * ret_chunkwise_states: from k, v and the decays, writes into `workspace` the
+ *   state entering every chunk (slot i = R_{i-1}; slot 0 = state_in when
+ *   given) and, when state_out is not NULL, the final float32 state.  It
+ *   launches nothing when there is a single chunk and no state enters or
+ *   leaves.  Arguments as for ret_chunkwise.
+ * ret_chunkwise_output: from q, k, v, the decays and the workspace that
+ *   ret_chunkwise_states wrote with the same B, H, N, dk, dv, chunk and dtype,
+ *   writes o (with the fused GroupNorm when gn_eps >= 0).  has_state_in must
+ *   say whether that states call was given a state_in.  The workspace is
+ *   only read.
+ * The workspace layout is internal to the library and differs between the
+ * tensor-core and the other paths; nothing but these two calls may read or
+ * write it.  Errors as for ret_chunkwise; N == 0 writes nothing (the states
+ * call still copies or zeroes state_out).
+ */
+RET_API int ret_chunkwise_states(const void* k, const void* v, const float* gammas, int chunk,
+                         const float* state_in, float* state_out,
+                         int B, int H, int N, int dk, int dv, int dtype,
+                         void* workspace, size_t workspace_bytes, void* stream);
+RET_API int ret_chunkwise_output(const void* q, const void* k, const void* v, const float* gammas,
+                         int chunk, int has_state_in, void* o,
+                         int B, int H, int N, int dk, int dv, int dtype, float gn_eps,
+                         const void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device scratch compiled into the library for ret_chunkwise_noalloc. */
 #define RET_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 

@@ -28,6 +28,9 @@ SIGNATURES = {
     "ret_chunkwise": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P, _S, _P]),
     "ret_chunkwise_noalloc": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F,
                                    _P]),
+    "ret_chunkwise_states": (_I, [_P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _P, _S, _P]),
+    "ret_chunkwise_output": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P, _S,
+                                  _P]),
     "ret_step": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "ret_status_string": (ctypes.c_char_p, [_I]),
     "ret_last_cuda_error": (_I, []),
@@ -171,13 +174,7 @@ def chunkwise(q, k, v, gammas, chunk, state_in=None, state_out=None, return_stat
     if out is None:
         out = torch.empty((B, H, N, dv), dtype=q.dtype, device=dev)
     _check(out, "out", dtype=q.dtype, shape=(B, H, N, dv), device=dev)
-    need = chunkwise_workspace_bytes(B, H, N, dk, dv, chunk, q.dtype)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
-    ws_bytes = 0
-    if workspace is not None:
-        _check(workspace, "workspace", device=dev)
-        ws_bytes = workspace.numel() * workspace.element_size()
+    workspace, ws_bytes = _workspace(workspace, B, H, N, dk, dv, chunk, q.dtype, dev)
     eps = -1.0 if gn_eps is None else float(gn_eps)
     s = load_library().ret_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), int(chunk),
                                      _ptr(state_in), _ptr(state_out), _ptr(out),
@@ -187,6 +184,59 @@ def chunkwise(q, k, v, gammas, chunk, state_in=None, state_out=None, return_stat
         _raise("ret_chunkwise", s)
     if state_out is not None:
         return out, state_out
+    return out
+
+
+def _workspace(workspace, B, H, N, dk, dv, chunk, dtype, dev):
+    torch = _torch()
+    need = chunkwise_workspace_bytes(B, H, N, dk, dv, chunk, dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0
+    if workspace is not None:
+        _check(workspace, "workspace", device=dev)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    return workspace, ws_bytes
+
+
+def chunkwise_states(k, v, gammas, chunk, workspace, state_in=None, state_out=None):
+    """First phase of the chunkwise form (ret_chunkwise_states): the state
+    entering every chunk into `workspace` (uint8 CUDA tensor of at least
+    chunkwise_workspace_bytes()), and the final state into state_out if given."""
+    torch = _torch()
+    B, H, N, dk, dv, dev = _seq_args(k, k, v, gammas)
+    sshape = (B, H, dk, dv)
+    if state_in is not None:
+        _check(state_in, "state_in", dtype=torch.float32, shape=sshape, device=dev)
+    if state_out is not None:
+        _check(state_out, "state_out", dtype=torch.float32, shape=sshape, device=dev)
+    workspace, ws_bytes = _workspace(workspace, B, H, N, dk, dv, chunk, k.dtype, dev)
+    s = load_library().ret_chunkwise_states(_ptr(k), _ptr(v), _ptr(gammas), int(chunk),
+                                            _ptr(state_in), _ptr(state_out), B, H, N, dk, dv,
+                                            _dtype_code(k), _ptr(workspace), ws_bytes,
+                                            _stream(dev))
+    if s != RET_OK:
+        _raise("ret_chunkwise_states", s)
+    return workspace
+
+
+def chunkwise_output(q, k, v, gammas, chunk, workspace, has_state_in=False, gn_eps=None,
+                     out=None):
+    """Second phase of the chunkwise form (ret_chunkwise_output): o from the
+    workspace that chunkwise_states wrote for the same sizes; returns o."""
+    torch = _torch()
+    B, H, N, dk, dv, dev = _seq_args(q, k, v, gammas)
+    if out is None:
+        out = torch.empty((B, H, N, dv), dtype=q.dtype, device=dev)
+    _check(out, "out", dtype=q.dtype, shape=(B, H, N, dv), device=dev)
+    workspace, ws_bytes = _workspace(workspace, B, H, N, dk, dv, chunk, q.dtype, dev)
+    eps = -1.0 if gn_eps is None else float(gn_eps)
+    s = load_library().ret_chunkwise_output(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), int(chunk),
+                                            1 if has_state_in else 0, _ptr(out), B, H, N, dk, dv,
+                                            _dtype_code(q), eps, _ptr(workspace), ws_bytes,
+                                            _stream(dev))
+    if s != RET_OK:
+        _raise("ret_chunkwise_output", s)
     return out
 
 

@@ -98,50 +98,102 @@ size_t ret_chunkwise_workspace(int B, int H, int N, int dk, int dv, int chunk, i
   return ret::simt_workspace_bytes(B, H, N, dk, dv, chunk);
 }
 
-int ret_chunkwise(const void* q, const void* k, const void* v, const float* gammas, int chunk,
-                  const float* state_in, float* state_out, void* o, int B, int H, int N, int dk,
-                  int dv, int dtype, float gn_eps, void* workspace, size_t workspace_bytes,
-                  void* stream) {
+}  // extern "C"
+
+namespace {
+
+bool tc_config(int dtype, int dk, int dv, int chunk) {
+  return dtype == RET_BF16 && tc_dims(dk, dv) && tc_chunk(chunk);
+}
+
+// Checks shared by the chunkwise entry points (everything but the pointers
+// that only one phase reads).
+int check_chunkwise(int B, int H, int N, int dk, int dv, int dtype, int chunk,
+                    const float* gammas, const void* workspace, size_t workspace_bytes) {
   int s = check_seq_dims(B, H, N, dk, dv, dtype);
   if (s) return s;
-  if ((s = check_eps(gn_eps))) return s;
-  if (chunk < 1) return RET_EINVAL;
-  if (!gammas) return RET_EINVAL;
+  if (chunk < 1 || !gammas) return RET_EINVAL;
+  if (N == 0) return RET_OK;
+  const size_t need = ret_chunkwise_workspace(B, H, N, dk, dv, chunk, dtype);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return RET_EWORKSPACE;
+  if (workspace && !aligned16(workspace)) return RET_EINVAL;
+  if (tc_config(dtype, dk, dv, chunk)) {
+    const int nc = (N + chunk - 1) / chunk;
+    if ((int64_t)nc * (chunk / 128) > 65535) return RET_EUNSUPPORTED;
+  }
+  return RET_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ret_chunkwise_states(const void* k, const void* v, const float* gammas, int chunk,
+                         const float* state_in, float* state_out, int B, int H, int N, int dk,
+                         int dv, int dtype, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  int s = check_chunkwise(B, H, N, dk, dv, dtype, chunk, gammas, workspace, workspace_bytes);
+  if (s) return s;
   if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
     return RET_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t state_bytes = sizeof(float) * (size_t)B * H * dk * dv;
   if (N == 0) {
     // No tokens: the final state is the initial one.
-    if (!state_out) return RET_OK;
-    if (state_in == state_out) return RET_OK;
+    if (!state_out || state_in == state_out) return RET_OK;
+    const size_t state_bytes = sizeof(float) * (size_t)B * H * dk * dv;
     if (state_in)
       return cuda_status(
           cudaMemcpyAsync(state_out, state_in, state_bytes, cudaMemcpyDeviceToDevice, st));
     return cuda_status(cudaMemsetAsync(state_out, 0, state_bytes, st));
   }
+  if (!k || !v || !aligned16(k) || !aligned16(v)) return RET_EINVAL;
+  if (tc_config(dtype, dk, dv, chunk)) {
+    // Needed whenever a state enters, crosses a chunk boundary or is
+    // returned; the incoming state is also stored in workspace slot 0.
+    const int nc = (N + chunk - 1) / chunk;
+    if (nc == 1 && !state_out && !state_in) return RET_OK;
+    return cuda_status(ret::launch_tc_state(k, v, gammas, chunk, state_in, state_out, workspace,
+                                            state_in != nullptr, B, H, N, dk, dv, st));
+  }
+  return cuda_status(ret::launch_simt_states(k, v, gammas, chunk, state_in, state_out, B, H, N,
+                                             dk, dv, dtype, workspace, st));
+}
+
+int ret_chunkwise_output(const void* q, const void* k, const void* v, const float* gammas,
+                         int chunk, int has_state_in, void* o, int B, int H, int N, int dk, int dv,
+                         int dtype, float gn_eps, const void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  int s = check_chunkwise(B, H, N, dk, dv, dtype, chunk, gammas, workspace, workspace_bytes);
+  if (s) return s;
+  if ((s = check_eps(gn_eps))) return s;
+  if (N == 0) return RET_OK;
   if (!q || !k || !v || !o) return RET_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_EINVAL;
-  const size_t need = ret_chunkwise_workspace(B, H, N, dk, dv, chunk, dtype);
-  if (need > 0 && (!workspace || workspace_bytes < need)) return RET_EWORKSPACE;
-  if (workspace && !aligned16(workspace)) return RET_EINVAL;
-  if (dtype == RET_BF16 && tc_dims(dk, dv) && tc_chunk(chunk)) {
-    const int nc = (N + chunk - 1) / chunk;
-    if ((int64_t)nc * (chunk / 128) > 65535) return RET_EUNSUPPORTED;
-    // The state kernel runs whenever a state enters, crosses a chunk boundary
-    // or is returned; it also stores the incoming state in workspace slot 0.
-    if (nc > 1 || state_out || state_in) {
-      int s2 = cuda_status(ret::launch_tc_state(k, v, gammas, chunk, state_in, state_out,
-                                                workspace, state_in != nullptr, B, H, N, dk, dv,
-                                                st));
-      if (s2) return s2;
-    }
-    return cuda_status(ret::launch_tc_out(q, k, v, gammas, chunk, workspace,
-                                          state_in != nullptr, o, B, H, N, dk, dv, gn_eps, 0,
-                                          st));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tc_config(dtype, dk, dv, chunk))
+    return cuda_status(ret::launch_tc_out(q, k, v, gammas, chunk, workspace, has_state_in != 0, o,
+                                          B, H, N, dk, dv, gn_eps, 0, st));
+  return cuda_status(ret::launch_simt_output(q, k, v, gammas, chunk, o, B, H, N, dk, dv, dtype,
+                                             gn_eps, workspace, st));
+}
+
+int ret_chunkwise(const void* q, const void* k, const void* v, const float* gammas, int chunk,
+                  const float* state_in, float* state_out, void* o, int B, int H, int N, int dk,
+                  int dv, int dtype, float gn_eps, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  // Every check of both phases runs before the first launch.
+  int s = check_chunkwise(B, H, N, dk, dv, dtype, chunk, gammas, workspace, workspace_bytes);
+  if (s) return s;
+  if ((s = check_eps(gn_eps))) return s;
+  if (N > 0) {
+    if (!q || !k || !v || !o) return RET_EINVAL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_EINVAL;
   }
-  return cuda_status(ret::launch_simt_chunkwise(q, k, v, gammas, chunk, state_in, state_out, o,
-                                                B, H, N, dk, dv, dtype, gn_eps, workspace, st));
+  s = ret_chunkwise_states(k, v, gammas, chunk, state_in, state_out, B, H, N, dk, dv, dtype,
+                           workspace, workspace_bytes, stream);
+  if (s) return s;
+  return ret_chunkwise_output(q, k, v, gammas, chunk, state_in != nullptr, o, B, H, N, dk, dv,
+                              dtype, gn_eps, workspace, workspace_bytes, stream);
 }
 
 int ret_step(const void* q, const void* k, const void* v, const float* gammas, float* state,

@@ -12,10 +12,14 @@ cudaError_t launch_step(const void* q, const void* k, const void* v, const float
 
 size_t simt_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk);
 
-cudaError_t launch_simt_chunkwise(const void* q, const void* k, const void* v,
-                                  const float* gammas, int chunk, const float* state_in,
-                                  float* state_out, void* o, int B, int H, int N, int dk, int dv,
-                                  int dtype, float eps, void* ws, cudaStream_t st);
+// The chunkwise form on the SIMT cores, in its two phases: the float32 chunk
+// states into ws, then the outputs from them.
+cudaError_t launch_simt_states(const void* k, const void* v, const float* gammas, int chunk,
+                               const float* state_in, float* state_out, int B, int H, int N,
+                               int dk, int dv, int dtype, void* ws, cudaStream_t st);
+cudaError_t launch_simt_output(const void* q, const void* k, const void* v, const float* gammas,
+                               int chunk, void* o, int B, int H, int N, int dk, int dv, int dtype,
+                               float eps, const void* ws, cudaStream_t st);
 
 cudaError_t launch_simt_parallel(const void* q, const void* k, const void* v, const float* gammas,
                                  void* o, int B, int H, int N, int dk, int dv, int dtype,

@@ -272,30 +272,41 @@ static cudaError_t launch_out(const void* q, const void* k, const void* v, const
 }
 
 template <typename T>
-static cudaError_t simt_chunkwise_t(const void* q, const void* k, const void* v,
-                                    const float* gammas, int chunk, const float* state_in,
-                                    float* state_out, void* o, int B, int H, int N, int dk,
-                                    int dv, float eps, void* ws, cudaStream_t st) {
-  float* rws = static_cast<float*>(ws);
+static cudaError_t simt_states_t(const void* k, const void* v, const float* gammas, int chunk,
+                                 const float* state_in, float* state_out, int B, int H, int N,
+                                 int dk, int dv, void* ws, cudaStream_t st) {
   dim3 g1(cdiv(dv, SC_T), cdiv(dk, SC_T), B * H);
   simt_state_scan<T><<<g1, 256, 0, st>>>(static_cast<const T*>(k), static_cast<const T*>(v),
-                                         gammas, chunk, state_in, state_out, rws, H, N, dk, dv);
-  cudaError_t e = cudaPeekAtLastError();
-  if (e != cudaSuccess) return e;
+                                         gammas, chunk, state_in, state_out,
+                                         static_cast<float*>(ws), H, N, dk, dv);
+  return cudaPeekAtLastError();
+}
+
+template <typename T>
+static cudaError_t simt_output_t(const void* q, const void* k, const void* v, const float* gammas,
+                                 int chunk, void* o, int B, int H, int N, int dk, int dv,
+                                 float eps, const void* ws, cudaStream_t st) {
+  const float* rws = static_cast<const float*>(ws);
   if (eps >= 0.f)
     return launch_out<T, true>(q, k, v, gammas, chunk, rws, o, B, H, N, dk, dv, eps, st);
   return launch_out<T, false>(q, k, v, gammas, chunk, rws, o, B, H, N, dk, dv, eps, st);
 }
 
-cudaError_t launch_simt_chunkwise(const void* q, const void* k, const void* v,
-                                  const float* gammas, int chunk, const float* state_in,
-                                  float* state_out, void* o, int B, int H, int N, int dk, int dv,
-                                  int dtype, float eps, void* ws, cudaStream_t st) {
+cudaError_t launch_simt_states(const void* k, const void* v, const float* gammas, int chunk,
+                               const float* state_in, float* state_out, int B, int H, int N,
+                               int dk, int dv, int dtype, void* ws, cudaStream_t st) {
   if (dtype == RET_BF16)
-    return simt_chunkwise_t<__nv_bfloat16>(q, k, v, gammas, chunk, state_in, state_out, o, B, H,
-                                           N, dk, dv, eps, ws, st);
-  return simt_chunkwise_t<float>(q, k, v, gammas, chunk, state_in, state_out, o, B, H, N, dk, dv,
-                                 eps, ws, st);
+    return simt_states_t<__nv_bfloat16>(k, v, gammas, chunk, state_in, state_out, B, H, N, dk,
+                                        dv, ws, st);
+  return simt_states_t<float>(k, v, gammas, chunk, state_in, state_out, B, H, N, dk, dv, ws, st);
+}
+
+cudaError_t launch_simt_output(const void* q, const void* k, const void* v, const float* gammas,
+                               int chunk, void* o, int B, int H, int N, int dk, int dv, int dtype,
+                               float eps, const void* ws, cudaStream_t st) {
+  if (dtype == RET_BF16)
+    return simt_output_t<__nv_bfloat16>(q, k, v, gammas, chunk, o, B, H, N, dk, dv, eps, ws, st);
+  return simt_output_t<float>(q, k, v, gammas, chunk, o, B, H, N, dk, dv, eps, ws, st);
 }
 
 cudaError_t launch_simt_parallel(const void* q, const void* k, const void* v, const float* gammas,

@@ -19,9 +19,13 @@
 //   warps 2-5  decay mask: S_t -> registers -> P_t = S_t (.) D as bf16, written
 //              back into the first 64 columns of S_t's TMEM buffer; then
 //              Q (.) xi in place in the tile's Q buffer
-//   warps 6-9  epilogue: read O from TMEM, optional GroupNorm (Chan's merge of
-//              per-32-column statistics, one exchange with the peer CTA), bf16
-//              stores straight to global; frees O for the next tile's P V
+//   warps 6-   epilogue (4 warps, or with GroupNorm 8: two per TMEM lane
+//              quadrant, each on half of the columns): read O from TMEM,
+//              optional GroupNorm (Chan's merge of per-32-column statistics,
+//              of the two halves through shared memory, then one exchange
+//              with the peer CTA), bf16 rows staged in the tile's Q buffer and
+//              written by TMA; O is freed for the next tile's P V after the
+//              last TMEM read
 // The decay mask is never stored: each thread walks its row from the highest
 // column down, multiplying by gamma per column, one exp2 per 32 columns.
 // S_t's buffer is rewritten by Q K_{t+2}^T only after the MMA reading P_t was
@@ -57,7 +61,11 @@ template <int NQB> struct Layout {
   static constexpr int RING = (DATA_BYTES - NQB * QBUF) / STAGE;
   static constexpr int RING_OFF = NQB * QBUF;
 };
-constexpr int THREADS = 320;           // 10 warps
+// Epilogue warps: with GroupNorm (two passes over O and an exchange) two per
+// TMEM lane quadrant, each on half of the columns; without it one per quadrant
+// (more warps measured slower there).
+template <bool GN> constexpr int epi_warps() { return GN ? 8 : 4; }
+template <bool GN> constexpr int threads() { return (6 + epi_warps<GN>()) * 32; }
 
 struct Params {
   const float* gammas;
@@ -102,7 +110,27 @@ __device__ __forceinline__ void bulk_commit() {
 __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
-__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Named barriers of the epilogue warps (0 is __syncthreads).
+// Barrier 1 also ANDs a flag over the epilogue warps, so that they leave the
+// tile loop together when a wait has failed and never strand each other on a
+// named barrier.
+template <int EPI>
+__device__ __forceinline__ bool epi_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(EPI * 32)
+      : "memory");
+  return r != 0;
+}
+template <int EPI>
+__device__ __forceinline__ void epi_bar2() {
+  asm volatile("bar.sync 2, %0;" ::"n"(EPI * 32) : "memory");
+}
 
 __device__ __forceinline__ void chan_merge(float& n_a, float& mean_a, float& m2_a, float n_b,
                                            float mean_b, float m2_b) {
@@ -113,8 +141,21 @@ __device__ __forceinline__ void chan_merge(float& n_a, float& mean_a, float& m2_
   n_a = n;
 }
 
+// Sum of 32 values as a balanced tree: depth 5 instead of a 32-long chain.
+__device__ __forceinline__ float tree_sum32(const float (&x)[32]) {
+  float t[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) t[j] = x[j] + x[j + 16];
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+    for (int j = 0; j < w; ++j) t[j] += t[j + w];
+  }
+  return t[0];
+}
+
 template <bool GN, int NQB, int KQ>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(threads<GN>(), 1)
 chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_r,
              const __grid_constant__ CUtensorMap tm_o, const Params p) {
@@ -128,6 +169,8 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   uint8_t* smem = reinterpret_cast<uint8_t*>(aligned);
   constexpr int RING = Layout<NQB>::RING;
   constexpr int RING_OFF = Layout<NQB>::RING_OFF;
+  constexpr int EPI = epi_warps<GN>();
+  constexpr int NH = EPI / 4;          // epilogue warps per TMEM lane quadrant
   const int slice = blockIdx.x;
   const int c0 = slice * p.dvs;
   constexpr int kq = KQ;              // 64-wide blocks of d_k
@@ -167,7 +210,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     }
     mbar_init(qt_full, 4);
     mbar_init(o_full, 1);
-    mbar_init(o_free, 4);
+    mbar_init(o_free, EPI);
     mbar_init(drain, 1);
     fence_mbar_init();
   }
@@ -435,61 +478,81 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   } else {
     // ---------------- epilogue ----------------
     const int q = warp & 3;
+    const int half = (warp - 6) >> 2;     // which part of the slice's columns
     const int i = 32 * q + lane;
+    const int ncg = p.dvs / (32 * NH);    // 32-column groups per warp
+    const int cg0 = half * ncg;           // first group of this warp
     const uint32_t o_tm = tmem + (static_cast<uint32_t>(32 * q) << 16) + 256;
-    const int ncg = p.dvs / 32;
     int k = 0;
     bool ok = true;
     for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++k) {
       const Tile x = decode_tile(p, tile);
-      if (!mbar_wait(o_full, k & 1, 212)) { ok = false; break; }
+      const uint32_t stage_a = smem_u32(smem + Q_OFF + (k % NQB) * QBUF);
+      if (!epi_bar_and<EPI>(mbar_wait(o_full, k & 1, 212))) break;
       tc_fence_after();
       float mean = 0.f, inv = 1.f;
+      bool xok = true;
       if (GN) {
         float n_a = 0.f, m_a = 0.f, q_a = 0.f;
-        for (int cg = 0; cg < ncg; ++cg) {
+        for (int g = 0; g < ncg; ++g) {
           uint32_t v[32];
-          tmem_ld32(o_tm + 32 * cg, v);
+          tmem_ld32(o_tm + 32 * (cg0 + g), v);
           tmem_wait_ld();
-          float s1 = 0.f;
+          float d[32];
 #pragma unroll
-          for (int xx = 0; xx < 32; ++xx) s1 += __uint_as_float(v[xx]);
-          const float m = s1 * (1.f / 32.f);
-          float s2 = 0.f;
+          for (int xx = 0; xx < 32; ++xx) d[xx] = __uint_as_float(v[xx]);
+          const float m = tree_sum32(d) * (1.f / 32.f);
 #pragma unroll
-          for (int xx = 0; xx < 32; ++xx) {
-            const float d = __uint_as_float(v[xx]) - m;
-            s2 = fmaf(d, d, s2);
-          }
-          if (cg == 0) {
+          for (int xx = 0; xx < 32; ++xx) d[xx] = (d[xx] - m) * (d[xx] - m);
+          const float s2 = tree_sum32(d);
+          if (g == 0) {
             n_a = 32.f; m_a = m; q_a = s2;
           } else {
             chan_merge(n_a, m_a, q_a, 32.f, m, s2);
           }
         }
+        if (NH == 2) {
+          // the two halves of a row meet in shared memory (the tile's Q
+          // buffer, whose last reader, the inter-chunk MMA, is done); the
+          // second barrier keeps the staging writes below off it until both
+          // halves have read
+          float* part = reinterpret_cast<float*>(smem + Q_OFF + (k % NQB) * QBUF);
+          part[(2 * half) * 128 + i] = m_a;
+          part[(2 * half + 1) * 128 + i] = q_a;
+          epi_bar2<EPI>();
+          const float m_o = part[(2 * (half ^ 1)) * 128 + i];
+          const float q_o = part[(2 * (half ^ 1) + 1) * 128 + i];
+          epi_bar2<EPI>();
+          // merged in the same order by both halves: identical statistics
+          const float mb = half ? m_a : m_o, qb = half ? q_a : q_o;
+          if (half) { m_a = m_o; q_a = q_o; }
+          chan_merge(n_a, m_a, q_a, n_a, mb, qb);
+        }
         if (p.nslices > 1) {
           const int slot = k & 1;
           const uint32_t peer = static_cast<uint32_t>(slice ^ 1);
-          st_cluster_f32(&gn_red[slot * 256 + i], peer, m_a);
-          st_cluster_f32(&gn_red[slot * 256 + 128 + i], peer, q_a);
-          mbar_arrive_cluster(&gn_bar[slot], peer);
-          if (!mbar_wait_cluster(&gn_bar[slot], (k >> 1) & 1, 213)) { ok = false; }
+          if (half == 0) {
+            st_cluster_f32(&gn_red[slot * 256 + i], peer, m_a);
+            st_cluster_f32(&gn_red[slot * 256 + 128 + i], peer, q_a);
+            mbar_arrive_cluster(&gn_bar[slot], peer);
+          }
+          if (!mbar_wait_cluster(&gn_bar[slot], (k >> 1) & 1, 213)) { xok = false; }
           else chan_merge(n_a, m_a, q_a, static_cast<float>(p.dvs), gn_red[slot * 256 + i],
                           gn_red[slot * 256 + 128 + i]);
         }
         mean = m_a;
         inv = 1.0f / sqrtf(q_a / static_cast<float>(p.dv) + p.eps);
       }
-      // Stage bf16 O in this tile's Q buffer (its last reader, the inter-chunk
-      // MMA, is done) as [64-column block][128 rows][128 B] with the 128-byte
-      // swizzle, then write it with coalesced TMA stores; rows past N are
-      // clipped by the tensor map.
-      const uint32_t stage_a = smem_u32(smem + Q_OFF + (k % NQB) * QBUF) + i * 128;
-      for (int cg = 0; cg < ncg; ++cg) {
+      // Stage bf16 O in this tile's Q buffer as [64-column block][128 rows]
+      // [128 B] with the 128-byte swizzle, then write it with coalesced TMA
+      // stores; rows past N are clipped by the tensor map.
+      const uint32_t row_a = stage_a + i * 128;
+      for (int g = 0; g < ncg; ++g) {
+        const int cg = cg0 + g;
         uint32_t v[32];
         tmem_ld32(o_tm + 32 * cg, v);
         tmem_wait_ld();
-        if (cg == ncg - 1) {
+        if (g == ncg - 1) {
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(o_free);  // O may be overwritten now
@@ -499,7 +562,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         for (int xx = 0; xx < 16; ++xx)
           pk[xx] = pack_bf16((__uint_as_float(v[2 * xx]) - mean) * inv,
                              (__uint_as_float(v[2 * xx + 1]) - mean) * inv);
-        const uint32_t rowa = stage_a + (cg >> 1) * QBOX;
+        const uint32_t rowa = row_a + (cg >> 1) * QBOX;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int phys = (((cg & 1) * 4 + c) ^ (i & 7));
@@ -507,11 +570,10 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         }
       }
       fence_proxy_async_smem();
-      epi_bar();
+      ok = epi_bar_and<EPI>(xok);
       if (warp == 6 && lane == 0) {
-        const uint32_t sb = smem_u32(smem + Q_OFF + (k % NQB) * QBUF);
         for (int b = 0; b < p.dvs / 64; ++b)
-          tma_store_3d(&tm_o, sb + b * QBOX, c0 + b * 64, x.n0, x.bh);
+          tma_store_3d(&tm_o, stage_a + b * QBOX, c0 + b * 64, x.n0, x.bh);
         bulk_commit();
         bulk_wait_read0();
         mbar_arrive(&q_empty[k % NQB]);  // the loader may refill the buffer
@@ -578,7 +640,7 @@ cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const flo
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.nslices, nclusters, 1);
-  cfg.blockDim = dim3(THREADS);
+  cfg.blockDim = dim3(eps >= 0.f ? threads<true>() : threads<false>());
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];

@@ -36,14 +36,17 @@ namespace k2 {
 
 using namespace sm100;
 
-constexpr int T = 32;                  // tokens per stage
+#ifndef RET_K2_T
+#define RET_K2_T 32
+#endif
+constexpr int T = RET_K2_T;            // tokens per stage
 constexpr int NT = 128;                // state columns per CTA (d_v = 64 uses 64)
-constexpr int STAGES = 6;
-constexpr int BOX = T * 128;           // one [T][64] bf16 box: 4 KB
+constexpr int STAGES = 6 * 32 / T;     // 192 KB of stages
+constexpr int BOX = T * 128;           // one [T][64] bf16 box
 constexpr int K_OFF = 0;               // 4 boxes: up to 256 rows of d_k
 constexpr int V_OFF = 4 * BOX;         // 2 boxes: NT columns of V, becomes V hi
 constexpr int LO_OFF = 6 * BOX;        // 2 boxes
-constexpr int STAGE_BYTES = 8 * BOX;   // 32 KB
+constexpr int STAGE_BYTES = 8 * BOX;
 constexpr int BAR_OFF = STAGES * STAGE_BYTES;
 constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;
 constexpr int XF_WARPS = 8;            // V (.) zeta warps
@@ -192,18 +195,25 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         const uint32_t sb = smem_u32(smem + slot * STAGE_BYTES);
         const int j = j0 + row;
         const float z = (j < L) ? gpow(lg, L - 1 - j) : 0.f;
-        uint32_t off[2];
-        uint4 v[2];
+        constexpr int MAXP = T * (NT / 8) / NXT;  // chunks per thread at NT = 128
+        uint32_t off[MAXP];
+        uint4 v[MAXP];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < MAXP; ++u) {
           if (u < per) {
-            const int c = c_first + u;         // chunk within the row: box c/8, chunk c%8
+            // chunk within the row (box c/8, position c%8).  A 16-byte access
+            // is served a quarter warp at a time, and its eight threads own
+            // 8 * per consecutive chunks, so each 128-byte position occurs
+            // `per` times among them; rotating the order by the thread's rank
+            // among the threads sharing its positions makes every access of a
+            // quarter warp hit eight distinct positions: no bank conflicts
+            const int c = c_first + ((u + (((tt & 7) * per) >> 3)) & (per - 1));
             off[u] = (c >> 3) * BOX + row * 128 + (c & 7) * 16;
             v[u] = ld_shared_v4(sb + V_OFF + off[u]);
           }
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < MAXP; ++u) {
           if (u < per) {
             const uint32_t in[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
             uint32_t hi[4], lo[4];

@@ -110,3 +110,34 @@ def test_step_rejects_bad_arguments(lib):
     assert call(dv=2048) == ret.RET_EUNSUPPORTED
     assert call(dt=-1) == ret.RET_EINVAL
     assert call(eps=float("nan")) == ret.RET_EINVAL
+
+
+def test_chunkwise_phases_reject_bad_arguments(lib):
+    need = lib.ret_chunkwise_workspace(1, 2, 300, 64, 64, 64, 0)
+
+    def states(k=A, v=A, g=A, chunk=64, si=None, so=None, N=300, dt=0, ws=A, wsb=None):
+        wsb = need if wsb is None else wsb
+        return lib.ret_chunkwise_states(k, v, g, chunk, si, so, 1, 2, N, 64, 64, dt, ws, wsb,
+                                        None)
+
+    def output(q=A, k=A, v=A, g=A, chunk=64, hs=0, o=A, N=300, dt=0, eps=-1.0, ws=A, wsb=None):
+        wsb = need if wsb is None else wsb
+        return lib.ret_chunkwise_output(q, k, v, g, chunk, hs, o, 1, 2, N, 64, 64, dt, eps, ws,
+                                        wsb, None)
+
+    assert states(chunk=0) == ret.RET_EINVAL
+    assert states(g=None) == ret.RET_EINVAL
+    assert states(k=None) == ret.RET_EINVAL
+    assert states(so=M) == ret.RET_EINVAL
+    assert states(ws=None) == ret.RET_EWORKSPACE
+    assert states(wsb=need - 1) == ret.RET_EWORKSPACE
+    assert states(dt=3) == ret.RET_EINVAL
+    assert output(q=None) == ret.RET_EINVAL
+    assert output(o=M) == ret.RET_EINVAL
+    assert output(eps=float("nan")) == ret.RET_EINVAL
+    assert output(ws=None) == ret.RET_EWORKSPACE
+    assert output(ws=M) == ret.RET_EINVAL
+    # no tokens: the output phase writes nothing and the states phase has no
+    # state to copy
+    assert output(N=0, q=None, k=None, v=None, o=None, ws=None, wsb=0) == ret.RET_OK
+    assert states(N=0, k=None, v=None, ws=None, wsb=0) == ret.RET_OK

@@ -132,6 +132,29 @@ def test_chunkwise_without_state_out_and_in_place(torch_cuda, ret):
     assert _rel(s, s_ref) <= STATE_TOL
 
 
+@pytest.mark.parametrize("dt,chunk,gn", [("bf16", 256, 1e-5), ("f32", 100, None)])
+def test_chunkwise_in_two_phases(torch_cuda, ret, dt, chunk, gn):
+    """ret_chunkwise_states then ret_chunkwise_output: the oracle's result, and
+    bit for bit what the one-call form returns."""
+    torch = torch_cuda
+    B, H, N, dk, dv = 1, 2, 900, 128, 256
+    inp = wl.make_inputs(B, H, N, dk, dv, dt, seed=31, with_state=True)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    s0 = _dev(inp["state"])
+    ws = torch.empty(ret.chunkwise_workspace_bytes(B, H, N, dk, dv, chunk, q.dtype),
+                     dtype=torch.uint8, device="cuda")
+    s = torch.empty_like(s0)
+    ret.chunkwise_states(k, v, g, chunk, ws, state_in=s0, state_out=s)
+    o = ret.chunkwise_output(q, k, v, g, chunk, ws, has_state_in=True, gn_eps=gn)
+    o1, s1 = ret.chunkwise(q, k, v, g, chunk, state_in=s0, return_state=True, gn_eps=gn)
+    torch.cuda.synchronize()
+    o_ref, s_ref = _ref_chunkwise(inp, chunk, gn, True)
+    assert _rel(o, o_ref) <= TOL[dt]
+    assert _rel(s, s_ref) <= STATE_TOL
+    assert torch.equal(o, o1) and torch.equal(s, s1)
+
+
 # --- parallel form -----------------------------------------------------------------
 
 PAR_CASES = [
