@@ -154,6 +154,19 @@ __device__ __forceinline__ float tree_sum32(const float (&x)[32]) {
   return t[0];
 }
 
+// Sum of squares of 32 values, the same tree.
+__device__ __forceinline__ float tree_sumsq32(const float (&x)[32]) {
+  float t[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) t[j] = fmaf(x[j], x[j], x[j + 16] * x[j + 16]);
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+    for (int j = 0; j < w; ++j) t[j] += t[j + w];
+  }
+  return t[0];
+}
+
 template <bool GN, int NQB, int KQ>
 __global__ void __launch_bounds__(threads<GN>(), 1)
 chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -171,6 +184,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   constexpr int RING_OFF = Layout<NQB>::RING_OFF;
   constexpr int EPI = epi_warps<GN>();
   constexpr int NH = EPI / 4;          // epilogue warps per TMEM lane quadrant
+  constexpr int GN_G = DVS / (32 * NH);  // most 32-column groups an epilogue warp holds
   const int slice = blockIdx.x;
   const int c0 = slice * p.dvs;
   constexpr int kq = KQ;              // 64-wide blocks of d_k
@@ -490,25 +504,48 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       const uint32_t stage_a = smem_u32(smem + Q_OFF + (k % NQB) * QBUF);
       if (!epi_bar_and<EPI>(mbar_wait(o_full, k & 1, 212))) break;
       tc_fence_after();
-      float mean = 0.f, inv = 1.f;
       bool xok = true;
+      const uint32_t row_a = stage_a + i * 128;
       if (GN) {
+        // One pass over O in TMEM: per 32-column group the mean m_g, the
+        // squared deviations (Chan's merge across groups) and the deviations
+        // x - m_g themselves, scaled by sc_g = 1 / rms(x - m_g) and kept in
+        // registers as f16 (11-bit significands at unit scale, so the error
+        // stays below the bf16 rounding of the output).  O is released right
+        // after the last load; the exchanges and the normalisation
+        //     y = (x - m_g) sc_g (inv / sc_g) + (m_g - mean) inv
+        // run from registers while the next tile's P V proceeds.
+        uint32_t hv[GN_G][16];
+        float gm[GN_G], gs[GN_G];
         float n_a = 0.f, m_a = 0.f, q_a = 0.f;
-        for (int g = 0; g < ncg; ++g) {
-          uint32_t v[32];
-          tmem_ld32(o_tm + 32 * (cg0 + g), v);
-          tmem_wait_ld();
-          float d[32];
 #pragma unroll
-          for (int xx = 0; xx < 32; ++xx) d[xx] = __uint_as_float(v[xx]);
-          const float m = tree_sum32(d) * (1.f / 32.f);
+        for (int g = 0; g < GN_G; ++g) {
+          if (g < ncg) {
+            uint32_t v[32];
+            tmem_ld32(o_tm + 32 * (cg0 + g), v);
+            tmem_wait_ld();
+            if (g == ncg - 1) {
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(o_free);  // O may be overwritten now
+            }
+            float d[32];
 #pragma unroll
-          for (int xx = 0; xx < 32; ++xx) d[xx] = (d[xx] - m) * (d[xx] - m);
-          const float s2 = tree_sum32(d);
-          if (g == 0) {
-            n_a = 32.f; m_a = m; q_a = s2;
-          } else {
-            chan_merge(n_a, m_a, q_a, 32.f, m, s2);
+            for (int xx = 0; xx < 32; ++xx) d[xx] = __uint_as_float(v[xx]);
+            const float m = tree_sum32(d) * (1.f / 32.f);
+#pragma unroll
+            for (int xx = 0; xx < 32; ++xx) d[xx] -= m;
+            const float s2 = tree_sumsq32(d);
+            const float sc = s2 > 0.f ? rsqrtf(s2 * (1.f / 32.f)) : 1.f;
+#pragma unroll
+            for (int xx = 0; xx < 16; ++xx) hv[g][xx] = pack_f16(d[2 * xx] * sc, d[2 * xx + 1] * sc);
+            gm[g] = m;
+            gs[g] = sc;
+            if (g == 0) {
+              n_a = 32.f; m_a = m; q_a = s2;
+            } else {
+              chan_merge(n_a, m_a, q_a, 32.f, m, s2);
+            }
           }
         }
         if (NH == 2) {
@@ -540,33 +577,51 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           else chan_merge(n_a, m_a, q_a, static_cast<float>(p.dvs), gn_red[slot * 256 + i],
                           gn_red[slot * 256 + 128 + i]);
         }
-        mean = m_a;
-        inv = 1.0f / sqrtf(q_a / static_cast<float>(p.dv) + p.eps);
-      }
-      // Stage bf16 O in this tile's Q buffer as [64-column block][128 rows]
-      // [128 B] with the 128-byte swizzle, then write it with coalesced TMA
-      // stores; rows past N are clipped by the tensor map.
-      const uint32_t row_a = stage_a + i * 128;
-      for (int g = 0; g < ncg; ++g) {
-        const int cg = cg0 + g;
-        uint32_t v[32];
-        tmem_ld32(o_tm + 32 * cg, v);
-        tmem_wait_ld();
-        if (g == ncg - 1) {
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(o_free);  // O may be overwritten now
+        const float inv = 1.0f / sqrtf(q_a / static_cast<float>(p.dv) + p.eps);
+#pragma unroll
+        for (int g = 0; g < GN_G; ++g) {
+          if (g < ncg) {
+            const int cg = cg0 + g;
+            const float a = inv / gs[g];
+            const float b = (gm[g] - m_a) * inv;
+            uint32_t pk[16];
+#pragma unroll
+            for (int xx = 0; xx < 16; ++xx)
+              pk[xx] = pack_bf16(fmaf(f16lo_to_f32(hv[g][xx]), a, b),
+                                 fmaf(f16hi_to_f32(hv[g][xx]), a, b));
+            const uint32_t rowa = row_a + (cg >> 1) * QBOX;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const int phys = (((cg & 1) * 4 + c) ^ (i & 7));
+              st_shared_v4(rowa + phys * 16, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
+                           pk[4 * c + 3]);
+            }
+          }
         }
-        uint32_t pk[16];
+      } else {
+        // Stage bf16 O in this tile's Q buffer as [64-column block][128 rows]
+        // [128 B] with the 128-byte swizzle, then write it with coalesced TMA
+        // stores; rows past N are clipped by the tensor map.
+        for (int g = 0; g < ncg; ++g) {
+          const int cg = cg0 + g;
+          uint32_t v[32];
+          tmem_ld32(o_tm + 32 * cg, v);
+          tmem_wait_ld();
+          if (g == ncg - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(o_free);  // O may be overwritten now
+          }
+          uint32_t pk[16];
 #pragma unroll
-        for (int xx = 0; xx < 16; ++xx)
-          pk[xx] = pack_bf16((__uint_as_float(v[2 * xx]) - mean) * inv,
-                             (__uint_as_float(v[2 * xx + 1]) - mean) * inv);
-        const uint32_t rowa = row_a + (cg >> 1) * QBOX;
+          for (int xx = 0; xx < 16; ++xx)
+            pk[xx] = pack_bf16(__uint_as_float(v[2 * xx]), __uint_as_float(v[2 * xx + 1]));
+          const uint32_t rowa = row_a + (cg >> 1) * QBOX;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int phys = (((cg & 1) * 4 + c) ^ (i & 7));
-          st_shared_v4(rowa + phys * 16, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          for (int c = 0; c < 4; ++c) {
+            const int phys = (((cg & 1) * 4 + c) ^ (i & 7));
+            st_shared_v4(rowa + phys * 16, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
         }
       }
       fence_proxy_async_smem();

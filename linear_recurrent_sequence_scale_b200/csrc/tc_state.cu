@@ -36,12 +36,10 @@ namespace k2 {
 
 using namespace sm100;
 
-#ifndef RET_K2_T
-#define RET_K2_T 32
-#endif
-constexpr int T = RET_K2_T;            // tokens per stage
+constexpr int T = 64;                  // tokens per stage (32 measured slower: more
+                                       // per-stage waits and fences per token)
 constexpr int NT = 128;                // state columns per CTA (d_v = 64 uses 64)
-constexpr int STAGES = 6 * 32 / T;     // 192 KB of stages
+constexpr int STAGES = 3;              // 3 x 64 KB
 constexpr int BOX = T * 128;           // one [T][64] bf16 box
 constexpr int K_OFF = 0;               // 4 boxes: up to 256 rows of d_k
 constexpr int V_OFF = 4 * BOX;         // 2 boxes: NT columns of V, becomes V hi
@@ -182,7 +180,7 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const int tt = threadIdx.x - 64;
     constexpr int NXT = XF_WARPS * 32;
     const int cpr = p.nt / 8;                  // 16-byte chunks per token row
-    const int per = (T * cpr) / NXT;           // chunks per thread: 2 (NT = 128) or 1
+    const int per = (T * cpr) / NXT;           // chunks per thread: 4 (NT = 128) or 2
     const int row = (tt * per) / cpr;
     const int c_first = (tt * per) % cpr;
     int g = 0;

@@ -98,6 +98,12 @@ def _as_dtype(x32: np.ndarray, dtype: str) -> Tensor:
     raise ValueError(dtype)
 
 
+def from_values(x, dtype: str) -> Tensor:
+    """A Tensor holding the given values, cast to float32 (and for bf16
+    rounded to nearest even)."""
+    return _as_dtype(np.asarray(x, dtype=np.float32), dtype)
+
+
 def draw(rng: np.random.Generator, shape, scale: float, dtype: str) -> Tensor:
     x = (rng.standard_normal(size=shape) * scale).astype(np.float32)
     return _as_dtype(x, dtype)

@@ -155,6 +155,30 @@ def test_chunkwise_in_two_phases(torch_cuda, ret, dt, chunk, gn):
     assert torch.equal(o, o1) and torch.equal(s, s1)
 
 
+def test_groupnorm_far_from_zero_mean(torch_cuda, ret):
+    """GroupNorm where every output row carries a large common offset and the
+    32-column groups differ in spread by 30x: the normalised deviations must
+    still come out to bf16 accuracy (chunkwise with two d_v slices, and the
+    parallel form with one)."""
+    torch = torch_cuda
+    B, H, N, dk, dv, C = 1, 2, 600, 128, 512, 256
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=41)
+    col = np.where((np.arange(dv) // 32) % 4 == 0, 30.0, 1.0)
+    v = wl.from_values(inp["v"].exact * col + 40.0, "bf16")
+    q, k, vd = _dev(inp["q"]), _dev(inp["k"]), _dev(v)
+    g = _gam(torch, inp["gammas"])
+    o = ret.chunkwise(q, k, vd, g, C, gn_eps=1e-5)
+    o_ref, _ = oracle.chunkwise(inp["q"].exact, inp["k"].exact, v.exact, inp["gammas"], C)
+    o_ref = oracle.group_norm(o_ref, 1e-5)
+    vs = vd[..., :256].contiguous()
+    op = ret.parallel(q, k, vs, g, gn_eps=1e-5)
+    p_ref, _ = oracle.parallel(inp["q"].exact, inp["k"].exact, v.exact[..., :256], inp["gammas"])
+    p_ref = oracle.group_norm(p_ref, 1e-5)
+    torch.cuda.synchronize()
+    assert _rel(o, o_ref) <= TOL["bf16"]
+    assert _rel(op, p_ref) <= TOL["bf16"]
+
+
 # --- parallel form -----------------------------------------------------------------
 
 PAR_CASES = [
