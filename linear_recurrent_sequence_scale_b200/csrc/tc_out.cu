@@ -50,7 +50,7 @@ constexpr int QBOX = 128 * 128;        // [128 rows][64] bf16 = 16 KB
 constexpr int VBOX = 64 * 128;         // [64 rows][64] bf16 = 8 KB
 constexpr int QBUF = 4 * QBOX;         // one Q tile, d_k <= 256
 constexpr int Q_OFF = 0;
-constexpr int DATA_BYTES = 7 * STAGE;  // Q buffers + ring: 2 Q + 3 stages, or 1 Q + 5 stages
+constexpr int DATA_BYTES = 7 * 32768;  // Q buffers + ring stages
 constexpr int GN_OFF = DATA_BYTES;     // [2 slots][2 values][128] floats
 constexpr int BAR_OFF = GN_OFF + 2048;
 constexpr int ALIGN_SLACK = 512;
@@ -60,7 +60,10 @@ constexpr int SMEM_BYTES = BAR_OFF + 256 + ALIGN_SLACK;
 template <int NQB> struct Layout {
   static constexpr int RING = (DATA_BYTES - NQB * QBUF) / STAGE;
   static constexpr int RING_OFF = NQB * QBUF;
+  static_assert(RING >= 2 && RING_OFF + RING * STAGE <= DATA_BYTES, "ring layout");
+  static_assert((2 * RING + 15) * 8 <= SMEM_BYTES - ALIGN_SLACK - BAR_OFF, "barrier area");
 };
+static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA");
 // Epilogue warps: with GroupNorm (two passes over O and an exchange) two per
 // TMEM lane quadrant, each on half of the columns; without it one per quadrant
 // (more warps measured slower there).
@@ -72,6 +75,7 @@ struct Params {
   __nv_bfloat16* o;
   int H, N, chunk, tpc, nc, dk, dv, dvs, nslices, ntiles;
   int chunked;     // 1: chunkwise form (R from the workspace), 0: parallel form
+  int grouped;     // 1: a CTA runs the row tiles of a chunk back to back
   int has_state0;  // workspace slot 0 holds an incoming state
   float eps;       // GroupNorm epsilon (< 0: none)
 };
@@ -93,6 +97,18 @@ __device__ __forceinline__ Tile decode_tile(const Params& p, int t) {
   x.nt = x.r + 1;
   x.has_r = p.chunked && (x.ci > 0 || p.has_state0);
   return x;
+}
+
+// The k-th work tile of this CTA (cluster row blockIdx.y of gridDim.y), or -1
+// past the end.  Grouped: whole chunks go round-robin over the cluster rows
+// and a CTA runs the row tiles of a chunk back to back (longest first), so
+// the K/V tiles and the chunk state its later row tiles re-read are still in
+// L2 from the first; otherwise (few chunks, e.g. the parallel form) single
+// tiles go round-robin.
+__device__ __forceinline__ int tile_at(const Params& p, int k) {
+  const int t = p.grouped ? (blockIdx.y + (k / p.tpc) * gridDim.y) * p.tpc + k % p.tpc
+                          : blockIdx.y + k * gridDim.y;
+  return t < p.ntiles ? t : -1;
 }
 
 // Chan et al.: merge (n_b, mean_b, m2_b) into (n_a, mean_a, m2_a).
@@ -237,8 +253,6 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   tc_fence_after();
   if (p.nslices > 1) cluster_sync_all();  // peer barriers exist before any remote arrive
   const uint32_t tmem = *tmem_slot;
-  const int tile0 = blockIdx.y;
-  const int tstep = gridDim.y;
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -256,8 +270,8 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       // that needs the Q starts.
       int qn = 0;  // next Q to load (tile sequence number)
       auto issue_q = [&](bool block) -> bool {
-        const int tile = tile0 + qn * tstep;
-        if (tile >= p.ntiles || qn > k + (NQB - 1)) return true;
+        const int tile = tile_at(p, qn);
+        if (tile < 0 || qn > k + (NQB - 1)) return true;
         const int qb = qn % NQB;
         const uint32_t par = ((qn / NQB) & 1) ^ 1;
         if (block) {
@@ -280,7 +294,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         mbar_arrive_expect_tx(bar, bytes);
         return smem + RING_OFF + slot * STAGE;
       };
-      for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++k) {
+      for (int tile = tile_at(p, k); tile >= 0 && ok; tile = tile_at(p, ++k)) {
         const Tile x = decode_tile(p, tile);
         while (ok && qn <= k) ok = issue_q(true);  // this tile's own Q
         for (int t = 0; t <= x.nt && ok; ++t) {
@@ -343,7 +357,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       // Descriptors: one full descriptor per operand buffer, then constant
       // offsets (the start address sits in the low bits, in 16-byte units), so
       // the issuing thread spends its time on MMAs, not on address arithmetic.
-      for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++k) {
+      for (int tile = tile_at(p, k); tile >= 0 && ok; tile = tile_at(p, ++k)) {
         const Tile x = decode_tile(p, tile);
         const int qb = k % NQB;
         const uint64_t qd = sdesc_sw128(smem_u32(smem + Q_OFF + qb * QBUF), 16, 1024);
@@ -424,7 +438,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
     int sc = 0, k = 0;
     bool ok = true;
-    for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++k) {
+    for (int tile = tile_at(p, k); tile >= 0 && ok; tile = tile_at(p, ++k)) {
       const Tile x = decode_tile(p, tile);
       const int h = x.bh % p.H;
       const float gam = p.gammas[h];
@@ -499,7 +513,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     const uint32_t o_tm = tmem + (static_cast<uint32_t>(32 * q) << 16) + 256;
     int k = 0;
     bool ok = true;
-    for (int tile = tile0; tile < p.ntiles && ok; tile += tstep, ++k) {
+    for (int tile = tile_at(p, k); tile >= 0 && ok; tile = tile_at(p, ++k)) {
       const Tile x = decode_tile(p, tile);
       const uint32_t stage_a = smem_u32(smem + Q_OFF + (k % NQB) * QBUF);
       if (!epi_bar_and<EPI>(mbar_wait(o_full, k & 1, 212))) break;
@@ -672,6 +686,7 @@ cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const flo
   const int64_t ntiles = (int64_t)BH * p.nc * p.tpc;
   if (ntiles > (int64_t)1 << 30) return cudaErrorInvalidConfiguration;
   p.ntiles = static_cast<int>(ntiles);
+  p.grouped = 0;
 
   int dev = 0, nsm = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -681,6 +696,7 @@ cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const flo
   int nclusters = nsm / p.nslices;
   if (nclusters > p.ntiles) nclusters = p.ntiles;
   if (nclusters < 1) nclusters = 1;
+  p.grouped = p.tpc > 1 && ntiles / p.tpc >= 4 * nclusters;
 
   CUtensorMap tm_q, tm_k, tm_v, tm_r, tm_o;
   if ((e = make_tmap_bf16_3d(&tm_q, q, dk, N, BH, 64, BM)) != cudaSuccess) return e;
