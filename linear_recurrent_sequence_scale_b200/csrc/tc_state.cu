@@ -48,6 +48,15 @@ constexpr int STAGE_BYTES = 8 * BOX;
 constexpr int BAR_OFF = STAGES * STAGE_BYTES;
 constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;
 constexpr int XF_WARPS = 8;            // V (.) zeta warps
+#ifndef RET_K2_XG
+#define RET_K2_XG 1
+#endif
+constexpr int XG = RET_K2_XG;          // groups of transform warps, taking stages in turn
+constexpr int XG_THREADS = XF_WARPS * 32 / XG;
+// Each ring slot must belong to one group, so that a group waiting on a
+// slot's mbarrier is never more than one phase ahead of it (a parity wait
+// two phases ahead would pass at once).
+static_assert(XF_WARPS % XG == 0 && STAGES % XG == 0, "transform groups own whole ring slots");
 constexpr int EPI_WARP0 = 2 + XF_WARPS;  // first state warp
 constexpr int THREADS = (EPI_WARP0 + 8) * 32;  // 18 warps
 
@@ -91,7 +100,7 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&xf[s], XF_WARPS);
+      mbar_init(&xf[s], XF_WARPS / XG);
       mbar_init(&empty[s], 1);
     }
     mbar_init(h_full, 1);
@@ -177,10 +186,10 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     // A stage holds T token rows of NT columns (16-byte chunks, 8 per 64-column
     // box row).  Each thread owns consecutive chunks of one token row, so it
     // needs one zeta per stage and can issue all its loads before any store.
-    const int tt = threadIdx.x - 64;
-    constexpr int NXT = XF_WARPS * 32;
+    const int grp = (threadIdx.x - 64) / XG_THREADS;  // takes stages grp, grp + XG, ...
+    const int tt = (threadIdx.x - 64) % XG_THREADS;
     const int cpr = p.nt / 8;                  // 16-byte chunks per token row
-    const int per = (T * cpr) / NXT;           // chunks per thread: 4 (NT = 128) or 2
+    const int per = (T * cpr) / XG_THREADS;    // chunks per thread
     const int row = (tt * per) / cpr;
     const int c_first = (tt * per) % cpr;
     int g = 0;
@@ -188,12 +197,13 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     for (int ci = 0; ci < p.nc && ok; ++ci) {
       const int L = min(p.chunk, p.N - ci * p.chunk);
       for (int j0 = 0; j0 < L; j0 += T, ++g) {
+        if (g % XG != grp) continue;
         const int slot = g % STAGES;
         if (!mbar_wait(&full[slot], (g / STAGES) & 1, 104)) { ok = false; break; }
         const uint32_t sb = smem_u32(smem + slot * STAGE_BYTES);
         const int j = j0 + row;
         const float z = (j < L) ? gpow(lg, L - 1 - j) : 0.f;
-        constexpr int MAXP = T * (NT / 8) / NXT;  // chunks per thread at NT = 128
+        constexpr int MAXP = T * (NT / 8) / XG_THREADS;  // chunks per thread at NT = 128
         uint32_t off[MAXP];
         uint4 v[MAXP];
 #pragma unroll
