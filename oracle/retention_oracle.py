@@ -40,6 +40,8 @@ in the design notes):
     fix none of these conventions.
   * No scaling or normalising factors are applied to QK^T, D or their
     product (the Medium page mentions three such factors without formulas).
+  * Gate: the block's "swish gating" is read as swish(G) (.) Y with the gate
+    G supplied by the caller, swish(x) = x sigmoid(x).
 """
 from __future__ import annotations
 
@@ -157,6 +159,27 @@ def group_norm(o, eps: float):
     mu = o.mean(axis=-1, keepdims=True)
     var = ((o - mu) ** 2).mean(axis=-1, keepdims=True)
     return (o - mu) / np.sqrt(var + eps)
+
+
+def swish(x):
+    """swish(x) = x * sigmoid(x) = x / (1 + exp(-x)), the gate activation of
+    the retention block ([RetNet blog] core components, item 4: GroupNorm
+    with swish gating).  The pages name the activation only; this is its
+    standard definition, evaluated without overflow for large |x|."""
+    x = _f64(x)
+    e = np.exp(-np.abs(x))
+    sig = np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+    return x * sig
+
+
+def gated(y, g):
+    """Gated multi-scale retention output swish(G) (.) Y ([RetNet blog] core
+    components, item 4; abstract page, section 2.2 Gated Multi-Scale
+    Retention): Y is the retention output (after the per-head GroupNorm when
+    that is applied) and G a gate of the same shape.  Reading: G is an input
+    of the operator; the projection that produces it and the output
+    projection after the gate belong to the layer around it."""
+    return swish(g) * _f64(y)
 
 
 def rel_frobenius(x, ref) -> float:

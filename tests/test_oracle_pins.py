@@ -249,6 +249,51 @@ def test_msr_gammas_exact():
     assert np.all((g > 0) & (g < 1))
 
 
+# --- gate: swish(G) (.) Y ------------------------------------------------------
+
+def test_swish_identities():
+    """swish(x) - swish(-x) = x (sigmoid(x) + sigmoid(-x) = 1); swish(0) = 0;
+    sigmoid(ln 3) = 3/4, so swish(ln 3) = (3/4) ln 3; swish(x) -> x and
+    swish(-x) -> 0 as x grows; finite for |x| up to 1e4."""
+    x = np.linspace(-30.0, 30.0, 121)
+    np.testing.assert_allclose(oracle.swish(x) - oracle.swish(-x), x, rtol=0, atol=1e-12)
+    assert oracle.swish(0.0) == 0.0
+    assert abs(oracle.swish(np.log(3.0)) - 0.75 * np.log(3.0)) < 1e-15
+    assert abs(oracle.swish(40.0) - 40.0) < 1e-12
+    assert abs(oracle.swish(-40.0)) < 1e-14
+    assert np.all(np.isfinite(oracle.swish(np.array([-1e4, 1e4]))))
+
+
+def test_gated_pins():
+    """The gate multiplies element by element: G = ln 3 everywhere scales Y by
+    (3/4) ln 3; G = 0 gives 0; a gate of +40 on one column scales that column
+    by 40 (swish(x) -> x) and leaves the others at 0."""
+    rng = np.random.default_rng(21)
+    y = rng.standard_normal((2, 3, 5, 4))
+    np.testing.assert_allclose(oracle.gated(y, np.full_like(y, np.log(3.0))),
+                               0.75 * np.log(3.0) * y, rtol=1e-14)
+    assert np.all(oracle.gated(y, np.zeros_like(y)) == 0.0)
+    g = np.zeros_like(y)
+    g[..., 2] = 40.0
+    out = oracle.gated(y, g)
+    np.testing.assert_allclose(out[..., 2], 40.0 * y[..., 2], rtol=1e-12)
+    assert np.all(out[..., [0, 1, 3]] == 0.0)
+
+
+@pytest.mark.parametrize("mutation", ["sigmoid_only", "exp_sign", "tanh"])
+def test_gate_pins_catch_planted_mistakes(mutation):
+    x = np.linspace(-5.0, 5.0, 41)
+    if mutation == "sigmoid_only":
+        f = lambda t: 1.0 / (1.0 + np.exp(-t))
+    elif mutation == "exp_sign":
+        f = lambda t: t / (1.0 + np.exp(t))
+    else:
+        f = lambda t: t * np.tanh(t)
+    caught = (np.max(np.abs(f(x) - f(-x) - x)) > 1e-6
+              or abs(f(np.log(3.0)) - 0.75 * np.log(3.0)) > 1e-6)
+    assert caught
+
+
 # --- mutation tests: planted mistakes are caught by the pins --------------------
 
 def _chunkwise_mutant(q, k, v, gammas, chunk, mutation):
