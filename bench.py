@@ -22,6 +22,7 @@ is needed between steps.  The same line carries:
                 states so the 256 MB working set exceeds L2; % of measured HBM
   parallel      the parallel form on the 1.3B-class layer (8 x 8 heads x 2048)
   long_64k      chunkwise over 65536 tokens (1 x 16 heads)
+  gated         the headline step with the output gate swish(G) (.) GN(o)
   cpu_baseline  the float64 CPU oracle on a bounded sample of the same
                 workload (rank 0, N = 1 only)
 With N > 1 (torchrun) every rank runs the same per-GPU step on its own GPU
@@ -567,6 +568,29 @@ def run_ours(args):
                              "ms": cl * 1e3, "tflops": Fl / cl / 1e12,
                              "frac_tc": Fl / cl / 1e12 / peak}
         del ql, kl, vl, ol, sl, wsl
+        torch.cuda.empty_cache()
+
+        # ---------------- gated output on the headline workload ----------------
+        qg, kg, vg, gg = make_qkv(torch, w.B, w.H, w.N, w.dk, w.dv, device, seed=6000 + rank)
+        gate = torch.randn(vg.shape, device=device).bfloat16()
+        og = torch.empty_like(vg)
+        wsg = torch.empty(ret.chunkwise_workspace_bytes(w.B, w.H, w.N, w.dk, w.dv, w.chunk,
+                                                        torch.bfloat16),
+                          dtype=torch.uint8, device=device)
+        tg, _ = timed(lambda: ret.chunkwise(qg, kg, vg, gg, w.chunk, gn_eps=w.gn_eps, out=og,
+                                            workspace=wsg, gate=gate),
+                      sub_steps, 3, stream, device)
+        tu, _ = timed(lambda: ret.chunkwise(qg, kg, vg, gg, w.chunk, gn_eps=w.gn_eps, out=og,
+                                            workspace=wsg),
+                      sub_steps, 3, stream, device)
+        launches += 4 * sub_steps
+        cg_ = tg / sub_steps
+        extra["gated"] = {"workload": WORKLOAD + " with swish(gate) * GroupNorm(o)",
+                          "tokens_per_s": w.B * w.N / cg_, "ms": cg_ * 1e3,
+                          "ungated_ms": tu / sub_steps * 1e3,
+                          "tflops": F / cg_ / 1e12, "frac_tc": F / cg_ / 1e12 / peak,
+                          "gate_bytes": gate.numel() * gate.element_size()}
+        del qg, kg, vg, og, wsg, gate
         torch.cuda.empty_cache()
 
     # ---------------- CPU oracle baseline ----------------

@@ -173,6 +173,37 @@ RET_API int ret_chunkwise_noalloc(const void* q, const void* k, const void* v, c
 RET_API int ret_step(const void* q, const void* k, const void* v, const float* gammas, float* state,
              void* o, int B, int H, int dk, int dv, int dtype, float gn_eps, void* stream);
 
+/*
+ * Gated variants of the three forms ("RetNet - Retentive Network - A
+ * Successor to Transformer for LLMs", core components, item 4: GroupNorm with
+ * swish gating; abstract page, section 2.2 Gated Multi-Scale Retention):
+ *     o = swish(gate) (.) Y,   swish(x) = x / (1 + exp(-x)),
+ * where Y is what the ungated call writes (the retention output, after the
+ * per-head GroupNorm when gn_eps >= 0).  The gate is computed by the caller
+ * (the layer's gate projection); the output projection after it is not part
+ * of this library.
+ *   gate : same shape, layout and dtype as o ([B][H][N][dv], or [B][H][dv]
+ *          for the step), 16-byte aligned, only read; NULL gives exactly the
+ *          ungated call.
+ * Other arguments, results and errors as for the ungated call.  The gate is
+ * applied in the kernel that writes o (fused; no extra pass over o).
+ */
+RET_API int ret_parallel_gated(const void* q, const void* k, const void* v, const float* gammas,
+                       const void* gate, void* o, int B, int H, int N, int dk, int dv,
+                       int dtype, float gn_eps, void* stream);
+RET_API int ret_chunkwise_gated(const void* q, const void* k, const void* v, const float* gammas,
+                        int chunk, const float* state_in, float* state_out, const void* gate,
+                        void* o, int B, int H, int N, int dk, int dv, int dtype, float gn_eps,
+                        void* workspace, size_t workspace_bytes, void* stream);
+RET_API int ret_chunkwise_output_gated(const void* q, const void* k, const void* v,
+                               const float* gammas, int chunk, int has_state_in,
+                               const void* gate, void* o, int B, int H, int N, int dk, int dv,
+                               int dtype, float gn_eps, const void* workspace,
+                               size_t workspace_bytes, void* stream);
+RET_API int ret_step_gated(const void* q, const void* k, const void* v, const float* gammas,
+                   float* state, const void* gate, void* o, int B, int H, int dk, int dv,
+                   int dtype, float gn_eps, void* stream);
+
 /* Human-readable name of a ret_status value (static storage). */
 RET_API const char* ret_status_string(int status);
 

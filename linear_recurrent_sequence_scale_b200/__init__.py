@@ -32,6 +32,12 @@ SIGNATURES = {
     "ret_chunkwise_output": (_I, [_P, _P, _P, _P, _I, _I, _P, _I, _I, _I, _I, _I, _I, _F, _P, _S,
                                   _P]),
     "ret_step": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "ret_parallel_gated": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "ret_chunkwise_gated": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F,
+                                 _P, _S, _P]),
+    "ret_chunkwise_output_gated": (_I, [_P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I,
+                                        _F, _P, _S, _P]),
+    "ret_step_gated": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "ret_status_string": (ctypes.c_char_p, [_I]),
     "ret_last_cuda_error": (_I, []),
     "ret_version": (ctypes.c_char_p, []),
@@ -133,16 +139,29 @@ def _seq_args(q, k, v, gammas):
     return B, H, N, dk, dv, dev
 
 
-def parallel(q, k, v, gammas, gn_eps=None, out=None):
-    """Parallel form O = (Q K^T (.) D) V (ret_parallel); returns o."""
+def _gate(gate, like, shape, dev):
+    if gate is not None:
+        _check(gate, "gate", dtype=like.dtype, shape=shape, device=dev)
+    return gate
+
+
+def parallel(q, k, v, gammas, gn_eps=None, out=None, gate=None):
+    """Parallel form O = (Q K^T (.) D) V (ret_parallel); returns o.  With a
+    gate (same shape as o): o = swish(gate) * O (ret_parallel_gated)."""
     torch = _torch()
     B, H, N, dk, dv, dev = _seq_args(q, k, v, gammas)
     if out is None:
         out = torch.empty((B, H, N, dv), dtype=q.dtype, device=dev)
     _check(out, "out", dtype=q.dtype, shape=(B, H, N, dv), device=dev)
+    gate = _gate(gate, q, (B, H, N, dv), dev)
     eps = -1.0 if gn_eps is None else float(gn_eps)
-    s = load_library().ret_parallel(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), _ptr(out),
-                                    B, H, N, dk, dv, _dtype_code(q), eps, _stream(dev))
+    lib = load_library()
+    if gate is None:
+        s = lib.ret_parallel(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), _ptr(out),
+                             B, H, N, dk, dv, _dtype_code(q), eps, _stream(dev))
+    else:
+        s = lib.ret_parallel_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), _ptr(gate), _ptr(out),
+                                   B, H, N, dk, dv, _dtype_code(q), eps, _stream(dev))
     if s != RET_OK:
         _raise("ret_parallel", s)
     return out
@@ -155,12 +174,13 @@ def chunkwise_workspace_bytes(B, H, N, dk, dv, chunk, dtype) -> int:
 
 
 def chunkwise(q, k, v, gammas, chunk, state_in=None, state_out=None, return_state=False,
-              gn_eps=None, out=None, workspace=None):
-    """Chunkwise-recurrent form (ret_chunkwise).
+              gn_eps=None, out=None, workspace=None, gate=None):
+    """Chunkwise-recurrent form (ret_chunkwise; ret_chunkwise_gated with a gate).
 
     Returns o, or (o, state) when return_state is True or state_out is given.
     state_out may be the same tensor as state_in (updated in place).
     workspace: optional uint8 CUDA tensor of at least chunkwise_workspace_bytes().
+    gate: optional tensor shaped like o; o is then multiplied by swish(gate).
     """
     torch = _torch()
     B, H, N, dk, dv, dev = _seq_args(q, k, v, gammas)
@@ -174,12 +194,20 @@ def chunkwise(q, k, v, gammas, chunk, state_in=None, state_out=None, return_stat
     if out is None:
         out = torch.empty((B, H, N, dv), dtype=q.dtype, device=dev)
     _check(out, "out", dtype=q.dtype, shape=(B, H, N, dv), device=dev)
+    gate = _gate(gate, q, (B, H, N, dv), dev)
     workspace, ws_bytes = _workspace(workspace, B, H, N, dk, dv, chunk, q.dtype, dev)
     eps = -1.0 if gn_eps is None else float(gn_eps)
-    s = load_library().ret_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), int(chunk),
-                                     _ptr(state_in), _ptr(state_out), _ptr(out),
-                                     B, H, N, dk, dv, _dtype_code(q), eps,
-                                     _ptr(workspace), ws_bytes, _stream(dev))
+    lib = load_library()
+    if gate is None:
+        s = lib.ret_chunkwise(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), int(chunk),
+                              _ptr(state_in), _ptr(state_out), _ptr(out),
+                              B, H, N, dk, dv, _dtype_code(q), eps,
+                              _ptr(workspace), ws_bytes, _stream(dev))
+    else:
+        s = lib.ret_chunkwise_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), int(chunk),
+                                    _ptr(state_in), _ptr(state_out), _ptr(gate), _ptr(out),
+                                    B, H, N, dk, dv, _dtype_code(q), eps,
+                                    _ptr(workspace), ws_bytes, _stream(dev))
     if s != RET_OK:
         _raise("ret_chunkwise", s)
     if state_out is not None:
@@ -221,27 +249,37 @@ def chunkwise_states(k, v, gammas, chunk, workspace, state_in=None, state_out=No
 
 
 def chunkwise_output(q, k, v, gammas, chunk, workspace, has_state_in=False, gn_eps=None,
-                     out=None):
-    """Second phase of the chunkwise form (ret_chunkwise_output): o from the
-    workspace that chunkwise_states wrote for the same sizes; returns o."""
+                     out=None, gate=None):
+    """Second phase of the chunkwise form (ret_chunkwise_output, or
+    ret_chunkwise_output_gated with a gate): o from the workspace that
+    chunkwise_states wrote for the same sizes; returns o."""
     torch = _torch()
     B, H, N, dk, dv, dev = _seq_args(q, k, v, gammas)
     if out is None:
         out = torch.empty((B, H, N, dv), dtype=q.dtype, device=dev)
     _check(out, "out", dtype=q.dtype, shape=(B, H, N, dv), device=dev)
+    gate = _gate(gate, q, (B, H, N, dv), dev)
     workspace, ws_bytes = _workspace(workspace, B, H, N, dk, dv, chunk, q.dtype, dev)
     eps = -1.0 if gn_eps is None else float(gn_eps)
-    s = load_library().ret_chunkwise_output(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), int(chunk),
-                                            1 if has_state_in else 0, _ptr(out), B, H, N, dk, dv,
-                                            _dtype_code(q), eps, _ptr(workspace), ws_bytes,
-                                            _stream(dev))
+    lib = load_library()
+    if gate is None:
+        s = lib.ret_chunkwise_output(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), int(chunk),
+                                     1 if has_state_in else 0, _ptr(out), B, H, N, dk, dv,
+                                     _dtype_code(q), eps, _ptr(workspace), ws_bytes,
+                                     _stream(dev))
+    else:
+        s = lib.ret_chunkwise_output_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), int(chunk),
+                                           1 if has_state_in else 0, _ptr(gate), _ptr(out),
+                                           B, H, N, dk, dv, _dtype_code(q), eps,
+                                           _ptr(workspace), ws_bytes, _stream(dev))
     if s != RET_OK:
         _raise("ret_chunkwise_output", s)
     return out
 
 
-def step(q, k, v, gammas, state, gn_eps=None, out=None):
-    """One recurrent decode step (ret_step): state is updated in place; returns o.
+def step(q, k, v, gammas, state, gn_eps=None, out=None, gate=None):
+    """One recurrent decode step (ret_step; ret_step_gated with a gate [B,H,dv]):
+    state is updated in place; returns o.
     q, k [B,H,dk]; v [B,H,dv]; state [B,H,dk,dv] float32."""
     torch = _torch()
     if q.dim() != 3:
@@ -257,9 +295,15 @@ def step(q, k, v, gammas, state, gn_eps=None, out=None):
     if out is None:
         out = torch.empty((B, H, dv), dtype=q.dtype, device=dev)
     _check(out, "out", dtype=q.dtype, shape=(B, H, dv), device=dev)
+    gate = _gate(gate, q, (B, H, dv), dev)
     eps = -1.0 if gn_eps is None else float(gn_eps)
-    s = load_library().ret_step(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), _ptr(state), _ptr(out),
-                                B, H, dk, dv, _dtype_code(q), eps, _stream(dev))
+    lib = load_library()
+    if gate is None:
+        s = lib.ret_step(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), _ptr(state), _ptr(out),
+                         B, H, dk, dv, _dtype_code(q), eps, _stream(dev))
+    else:
+        s = lib.ret_step_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), _ptr(state), _ptr(gate),
+                               _ptr(out), B, H, dk, dv, _dtype_code(q), eps, _stream(dev))
     if s != RET_OK:
         _raise("ret_step", s)
     return out

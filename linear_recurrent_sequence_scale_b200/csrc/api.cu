@@ -72,22 +72,29 @@ int ret_device_error(void) {
   return a ? a : b;
 }
 
-int ret_parallel(const void* q, const void* k, const void* v, const float* gammas, void* o,
-                 int B, int H, int N, int dk, int dv, int dtype, float gn_eps, void* stream) {
+int ret_parallel_gated(const void* q, const void* k, const void* v, const float* gammas,
+                       const void* gate, void* o, int B, int H, int N, int dk, int dv, int dtype,
+                       float gn_eps, void* stream) {
   int s = check_seq_dims(B, H, N, dk, dv, dtype);
   if (s) return s;
   if ((s = check_eps(gn_eps))) return s;
   if (N == 0) return RET_OK;
   if (!q || !k || !v || !o || !gammas) return RET_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_EINVAL;
+  if (gate && !aligned16(gate)) return RET_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == RET_BF16 && tc_dims(dk, dv)) {
     if ((int64_t)((N + 127) / 128) > 65535) return RET_EUNSUPPORTED;
-    return cuda_status(ret::launch_tc_out(q, k, v, gammas, 0, nullptr, 0, o, B, H, N, dk, dv,
-                                          gn_eps, 1, st));
+    return cuda_status(ret::launch_tc_out(q, k, v, gammas, 0, nullptr, 0, gate, o, B, H, N, dk,
+                                          dv, gn_eps, 1, st));
   }
-  return cuda_status(ret::launch_simt_parallel(q, k, v, gammas, o, B, H, N, dk, dv, dtype,
+  return cuda_status(ret::launch_simt_parallel(q, k, v, gammas, gate, o, B, H, N, dk, dv, dtype,
                                                gn_eps, st));
+}
+
+int ret_parallel(const void* q, const void* k, const void* v, const float* gammas, void* o,
+                 int B, int H, int N, int dk, int dv, int dtype, float gn_eps, void* stream) {
+  return ret_parallel_gated(q, k, v, gammas, nullptr, o, B, H, N, dk, dv, dtype, gn_eps, stream);
 }
 
 size_t ret_chunkwise_workspace(int B, int H, int N, int dk, int dv, int chunk, int dtype) {
@@ -159,28 +166,37 @@ int ret_chunkwise_states(const void* k, const void* v, const float* gammas, int 
                                              dk, dv, dtype, workspace, st));
 }
 
-int ret_chunkwise_output(const void* q, const void* k, const void* v, const float* gammas,
-                         int chunk, int has_state_in, void* o, int B, int H, int N, int dk, int dv,
-                         int dtype, float gn_eps, const void* workspace, size_t workspace_bytes,
-                         void* stream) {
+int ret_chunkwise_output_gated(const void* q, const void* k, const void* v, const float* gammas,
+                               int chunk, int has_state_in, const void* gate, void* o, int B,
+                               int H, int N, int dk, int dv, int dtype, float gn_eps,
+                               const void* workspace, size_t workspace_bytes, void* stream) {
   int s = check_chunkwise(B, H, N, dk, dv, dtype, chunk, gammas, workspace, workspace_bytes);
   if (s) return s;
   if ((s = check_eps(gn_eps))) return s;
   if (N == 0) return RET_OK;
   if (!q || !k || !v || !o) return RET_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_EINVAL;
+  if (gate && !aligned16(gate)) return RET_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tc_config(dtype, dk, dv, chunk))
-    return cuda_status(ret::launch_tc_out(q, k, v, gammas, chunk, workspace, has_state_in != 0, o,
-                                          B, H, N, dk, dv, gn_eps, 0, st));
-  return cuda_status(ret::launch_simt_output(q, k, v, gammas, chunk, o, B, H, N, dk, dv, dtype,
-                                             gn_eps, workspace, st));
+    return cuda_status(ret::launch_tc_out(q, k, v, gammas, chunk, workspace, has_state_in != 0,
+                                          gate, o, B, H, N, dk, dv, gn_eps, 0, st));
+  return cuda_status(ret::launch_simt_output(q, k, v, gammas, chunk, gate, o, B, H, N, dk, dv,
+                                             dtype, gn_eps, workspace, st));
 }
 
-int ret_chunkwise(const void* q, const void* k, const void* v, const float* gammas, int chunk,
-                  const float* state_in, float* state_out, void* o, int B, int H, int N, int dk,
-                  int dv, int dtype, float gn_eps, void* workspace, size_t workspace_bytes,
-                  void* stream) {
+int ret_chunkwise_output(const void* q, const void* k, const void* v, const float* gammas,
+                         int chunk, int has_state_in, void* o, int B, int H, int N, int dk, int dv,
+                         int dtype, float gn_eps, const void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  return ret_chunkwise_output_gated(q, k, v, gammas, chunk, has_state_in, nullptr, o, B, H, N, dk,
+                                    dv, dtype, gn_eps, workspace, workspace_bytes, stream);
+}
+
+int ret_chunkwise_gated(const void* q, const void* k, const void* v, const float* gammas,
+                        int chunk, const float* state_in, float* state_out, const void* gate,
+                        void* o, int B, int H, int N, int dk, int dv, int dtype, float gn_eps,
+                        void* workspace, size_t workspace_bytes, void* stream) {
   // Every check of both phases runs before the first launch.
   int s = check_chunkwise(B, H, N, dk, dv, dtype, chunk, gammas, workspace, workspace_bytes);
   if (s) return s;
@@ -188,16 +204,28 @@ int ret_chunkwise(const void* q, const void* k, const void* v, const float* gamm
   if (N > 0) {
     if (!q || !k || !v || !o) return RET_EINVAL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RET_EINVAL;
+    if (gate && !aligned16(gate)) return RET_EINVAL;
   }
+  if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
+    return RET_EINVAL;
   s = ret_chunkwise_states(k, v, gammas, chunk, state_in, state_out, B, H, N, dk, dv, dtype,
                            workspace, workspace_bytes, stream);
   if (s) return s;
-  return ret_chunkwise_output(q, k, v, gammas, chunk, state_in != nullptr, o, B, H, N, dk, dv,
-                              dtype, gn_eps, workspace, workspace_bytes, stream);
+  return ret_chunkwise_output_gated(q, k, v, gammas, chunk, state_in != nullptr, gate, o, B, H, N,
+                                    dk, dv, dtype, gn_eps, workspace, workspace_bytes, stream);
 }
 
-int ret_step(const void* q, const void* k, const void* v, const float* gammas, float* state,
-             void* o, int B, int H, int dk, int dv, int dtype, float gn_eps, void* stream) {
+int ret_chunkwise(const void* q, const void* k, const void* v, const float* gammas, int chunk,
+                  const float* state_in, float* state_out, void* o, int B, int H, int N, int dk,
+                  int dv, int dtype, float gn_eps, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  return ret_chunkwise_gated(q, k, v, gammas, chunk, state_in, state_out, nullptr, o, B, H, N, dk,
+                             dv, dtype, gn_eps, workspace, workspace_bytes, stream);
+}
+
+int ret_step_gated(const void* q, const void* k, const void* v, const float* gammas,
+                   float* state, const void* gate, void* o, int B, int H, int dk, int dv,
+                   int dtype, float gn_eps, void* stream) {
   if (B < 1 || H < 1 || dk < 8 || dv < 8 || dk % 8 || dv % 8) return RET_EINVAL;
   if (!valid_dtype(dtype)) return RET_EINVAL;
   int s = check_eps(gn_eps);
@@ -206,9 +234,15 @@ int ret_step(const void* q, const void* k, const void* v, const float* gammas, f
   if (!q || !k || !v || !gammas || !state || !o) return RET_EINVAL;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(o))
     return RET_EINVAL;
+  if (gate && !aligned16(gate)) return RET_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return cuda_status(
-      ret::launch_step(q, k, v, gammas, state, o, B, H, dk, dv, dtype, gn_eps, st));
+      ret::launch_step(q, k, v, gammas, state, gate, o, B, H, dk, dv, dtype, gn_eps, st));
+}
+
+int ret_step(const void* q, const void* k, const void* v, const float* gammas, float* state,
+             void* o, int B, int H, int dk, int dv, int dtype, float gn_eps, void* stream) {
+  return ret_step_gated(q, k, v, gammas, state, nullptr, o, B, H, dk, dv, dtype, gn_eps, stream);
 }
 
 }  // extern "C"

@@ -53,4 +53,8 @@ __device__ __forceinline__ float gpow(float lg, int n) {
 
 __host__ __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
+// swish(x) = x sigmoid(x) = x / (1 + e^-x), the activation of the output
+// gate; e^-x overflows to inf for very negative x, which gives -0.
+__device__ __forceinline__ float swishf(float x) { return x / (1.0f + __expf(-x)); }
+
 }  // namespace ret

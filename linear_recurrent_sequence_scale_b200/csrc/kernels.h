@@ -6,9 +6,10 @@
 
 namespace ret {
 
+// gate (may be null): o is multiplied by swish(gate), same layout and type as o.
 cudaError_t launch_step(const void* q, const void* k, const void* v, const float* gammas,
-                        float* state, void* o, int B, int H, int dk, int dv, int dtype,
-                        float eps, cudaStream_t st);
+                        float* state, const void* gate, void* o, int B, int H, int dk, int dv,
+                        int dtype, float eps, cudaStream_t st);
 
 size_t simt_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk);
 
@@ -18,12 +19,12 @@ cudaError_t launch_simt_states(const void* k, const void* v, const float* gammas
                                const float* state_in, float* state_out, int B, int H, int N,
                                int dk, int dv, int dtype, void* ws, cudaStream_t st);
 cudaError_t launch_simt_output(const void* q, const void* k, const void* v, const float* gammas,
-                               int chunk, void* o, int B, int H, int N, int dk, int dv, int dtype,
-                               float eps, const void* ws, cudaStream_t st);
+                               int chunk, const void* gate, void* o, int B, int H, int N, int dk,
+                               int dv, int dtype, float eps, const void* ws, cudaStream_t st);
 
 cudaError_t launch_simt_parallel(const void* q, const void* k, const void* v, const float* gammas,
-                                 void* o, int B, int H, int N, int dk, int dv, int dtype,
-                                 float eps, cudaStream_t st);
+                                 const void* gate, void* o, int B, int H, int N, int dk, int dv,
+                                 int dtype, float eps, cudaStream_t st);
 
 }  // namespace ret
 
@@ -34,8 +35,9 @@ cudaError_t launch_tc_state(const void* k, const void* v, const float* gammas, i
                             const float* state_in, float* state_out, void* ws, int write_ws0,
                             int B, int H, int N, int dk, int dv, cudaStream_t st);
 cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const float* gammas,
-                          int chunk, const void* ws, int has_state0, void* o, int B, int H, int N,
-                          int dk, int dv, float eps, int parallel_form, cudaStream_t st);
+                          int chunk, const void* ws, int has_state0, const void* gate, void* o,
+                          int B, int H, int N, int dk, int dv, float eps, int parallel_form,
+                          cudaStream_t st);
 int tc_state_device_error();
 int tc_out_device_error();
 

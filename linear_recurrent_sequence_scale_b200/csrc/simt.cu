@@ -114,7 +114,8 @@ template <typename T, bool GN>
 __global__ void __launch_bounds__(256)
 simt_chunk_out(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                const float* __restrict__ gammas, int chunk, const float* __restrict__ rws,
-               T* __restrict__ o, int H, int N, int dk, int dv, float eps) {
+               const T* __restrict__ gate, T* __restrict__ o, int H, int N, int dk, int dv,
+               float eps) {
   extern __shared__ float sm[];
   const int ldq = dk + 1;
   float* qs = sm;                        // [CO_M][dk+1]
@@ -237,10 +238,11 @@ simt_chunk_out(const T* __restrict__ q, const T* __restrict__ k, const T* __rest
 
   if (row < nrows) {
     T* orow = o + ((size_t)bh * N + n0 + row) * dv;
+    const T* grow = gate ? gate + ((size_t)bh * N + n0 + row) * dv : nullptr;
 #pragma unroll
     for (int u = 0; u < CO_U; ++u) {
       const int c = cgp + 16 * u;
-      if (c < dv) Elem<T>::st(orow + c, acc[u]);
+      if (c < dv) Elem<T>::st(orow + c, grow ? acc[u] * swishf(Elem<T>::ld(grow + c)) : acc[u]);
     }
   }
 }
@@ -257,8 +259,8 @@ size_t simt_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk) {
 
 template <typename T, bool GN>
 static cudaError_t launch_out(const void* q, const void* k, const void* v, const float* gammas,
-                              int chunk, const float* rws, void* o, int B, int H, int N, int dk,
-                              int dv, float eps, cudaStream_t st) {
+                              int chunk, const float* rws, const void* gate, void* o, int B, int H,
+                              int N, int dk, int dv, float eps, cudaStream_t st) {
   const size_t smem = chunk_out_smem(dk, dv);
   auto fn = simt_chunk_out<T, GN>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -266,8 +268,8 @@ static cudaError_t launch_out(const void* q, const void* k, const void* v, const
   const int nc = cdiv(N, chunk);
   dim3 grid(nc * cdiv(chunk, CO_M), B * H);
   fn<<<grid, 256, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
-                              static_cast<const T*>(v), gammas, chunk, rws, static_cast<T*>(o), H,
-                              N, dk, dv, eps);
+                              static_cast<const T*>(v), gammas, chunk, rws,
+                              static_cast<const T*>(gate), static_cast<T*>(o), H, N, dk, dv, eps);
   return cudaPeekAtLastError();
 }
 
@@ -284,12 +286,12 @@ static cudaError_t simt_states_t(const void* k, const void* v, const float* gamm
 
 template <typename T>
 static cudaError_t simt_output_t(const void* q, const void* k, const void* v, const float* gammas,
-                                 int chunk, void* o, int B, int H, int N, int dk, int dv,
-                                 float eps, const void* ws, cudaStream_t st) {
+                                 int chunk, const void* gate, void* o, int B, int H, int N, int dk,
+                                 int dv, float eps, const void* ws, cudaStream_t st) {
   const float* rws = static_cast<const float*>(ws);
   if (eps >= 0.f)
-    return launch_out<T, true>(q, k, v, gammas, chunk, rws, o, B, H, N, dk, dv, eps, st);
-  return launch_out<T, false>(q, k, v, gammas, chunk, rws, o, B, H, N, dk, dv, eps, st);
+    return launch_out<T, true>(q, k, v, gammas, chunk, rws, gate, o, B, H, N, dk, dv, eps, st);
+  return launch_out<T, false>(q, k, v, gammas, chunk, rws, gate, o, B, H, N, dk, dv, eps, st);
 }
 
 cudaError_t launch_simt_states(const void* k, const void* v, const float* gammas, int chunk,
@@ -302,26 +304,27 @@ cudaError_t launch_simt_states(const void* k, const void* v, const float* gammas
 }
 
 cudaError_t launch_simt_output(const void* q, const void* k, const void* v, const float* gammas,
-                               int chunk, void* o, int B, int H, int N, int dk, int dv, int dtype,
-                               float eps, const void* ws, cudaStream_t st) {
+                               int chunk, const void* gate, void* o, int B, int H, int N, int dk,
+                               int dv, int dtype, float eps, const void* ws, cudaStream_t st) {
   if (dtype == RET_BF16)
-    return simt_output_t<__nv_bfloat16>(q, k, v, gammas, chunk, o, B, H, N, dk, dv, eps, ws, st);
-  return simt_output_t<float>(q, k, v, gammas, chunk, o, B, H, N, dk, dv, eps, ws, st);
+    return simt_output_t<__nv_bfloat16>(q, k, v, gammas, chunk, gate, o, B, H, N, dk, dv, eps, ws,
+                                        st);
+  return simt_output_t<float>(q, k, v, gammas, chunk, gate, o, B, H, N, dk, dv, eps, ws, st);
 }
 
 cudaError_t launch_simt_parallel(const void* q, const void* k, const void* v, const float* gammas,
-                                 void* o, int B, int H, int N, int dk, int dv, int dtype,
-                                 float eps, cudaStream_t st) {
+                                 const void* gate, void* o, int B, int H, int N, int dk, int dv,
+                                 int dtype, float eps, cudaStream_t st) {
   if (dtype == RET_BF16) {
     if (eps >= 0.f)
-      return launch_out<__nv_bfloat16, true>(q, k, v, gammas, N, nullptr, o, B, H, N, dk, dv,
-                                             eps, st);
-    return launch_out<__nv_bfloat16, false>(q, k, v, gammas, N, nullptr, o, B, H, N, dk, dv, eps,
-                                            st);
+      return launch_out<__nv_bfloat16, true>(q, k, v, gammas, N, nullptr, gate, o, B, H, N, dk,
+                                             dv, eps, st);
+    return launch_out<__nv_bfloat16, false>(q, k, v, gammas, N, nullptr, gate, o, B, H, N, dk,
+                                            dv, eps, st);
   }
   if (eps >= 0.f)
-    return launch_out<float, true>(q, k, v, gammas, N, nullptr, o, B, H, N, dk, dv, eps, st);
-  return launch_out<float, false>(q, k, v, gammas, N, nullptr, o, B, H, N, dk, dv, eps, st);
+    return launch_out<float, true>(q, k, v, gammas, N, nullptr, gate, o, B, H, N, dk, dv, eps, st);
+  return launch_out<float, false>(q, k, v, gammas, N, nullptr, gate, o, B, H, N, dk, dv, eps, st);
 }
 
 }  // namespace ret

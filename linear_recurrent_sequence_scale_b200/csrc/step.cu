@@ -42,8 +42,8 @@ __device__ __forceinline__ float block_sum_256(float x, float* scratch /* >= 8 f
 template <typename T, bool GN>
 __global__ void __launch_bounds__(STEP_THREADS)
 step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-            const float* __restrict__ gammas, float* __restrict__ state, T* __restrict__ o,
-            int H, int dk, int dv, float eps) {
+            const float* __restrict__ gammas, float* __restrict__ state,
+            const T* __restrict__ gate, T* __restrict__ o, int H, int dk, int dv, float eps) {
   extern __shared__ float smem[];
   float* qs = smem;                       // [dk]
   float* ks = smem + dk;                  // [dk]
@@ -125,17 +125,24 @@ step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
     float sq = 0.f;
     for (unsigned r = 0; r < nblk; ++r) sq += cluster.map_shared_rank(stats, r)[1];
     const float inv = 1.0f / sqrtf(sq / static_cast<float>(dv) + eps);
-    if (oval) Elem<T>::st(o + (size_t)bh * dv + oc, dev * inv);
+    if (oval) {
+      float y = dev * inv;
+      if (gate) y *= swishf(Elem<T>::ld(gate + (size_t)bh * dv + oc));
+      Elem<T>::st(o + (size_t)bh * dv + oc, y);
+    }
     cluster.sync();  // peers may still be reading this CTA's stats
   } else {
-    if (oval) Elem<T>::st(o + (size_t)bh * dv + oc, val);
+    if (oval) {
+      if (gate) val *= swishf(Elem<T>::ld(gate + (size_t)bh * dv + oc));
+      Elem<T>::st(o + (size_t)bh * dv + oc, val);
+    }
   }
 }
 
 template <typename T>
 static cudaError_t launch_step_t(const void* q, const void* k, const void* v, const float* gammas,
-                                 float* state, void* o, int B, int H, int dk, int dv, float eps,
-                                 cudaStream_t st) {
+                                 float* state, const void* gate, void* o, int B, int H, int dk,
+                                 int dv, float eps, cudaStream_t st) {
   const int nct = cdiv(dv, STEP_COLS);
   dim3 grid(nct, B * H);
   const size_t smem = sizeof(float) * (2 * dk + STEP_RG * STEP_COLS);
@@ -143,13 +150,14 @@ static cudaError_t launch_step_t(const void* q, const void* k, const void* v, co
   const T* kk = static_cast<const T*>(k);
   const T* vv = static_cast<const T*>(v);
   T* oo = static_cast<T*>(o);
+  const T* gg = static_cast<const T*>(gate);
   if (eps < 0.f) {
     auto fn = step_kernel<T, false>;
     if (smem > 48 * 1024) {
       cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
-    fn<<<grid, STEP_THREADS, smem, st>>>(qq, kk, vv, gammas, state, oo, H, dk, dv, eps);
+    fn<<<grid, STEP_THREADS, smem, st>>>(qq, kk, vv, gammas, state, gg, oo, H, dk, dv, eps);
     return cudaPeekAtLastError();
   }
   auto fn = step_kernel<T, true>;
@@ -169,15 +177,15 @@ static cudaError_t launch_step_t(const void* q, const void* k, const void* v, co
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, fn, qq, kk, vv, gammas, state, oo, H, dk, dv, eps);
+  return cudaLaunchKernelEx(&cfg, fn, qq, kk, vv, gammas, state, gg, oo, H, dk, dv, eps);
 }
 
 cudaError_t launch_step(const void* q, const void* k, const void* v, const float* gammas,
-                        float* state, void* o, int B, int H, int dk, int dv, int dtype,
-                        float eps, cudaStream_t st) {
+                        float* state, const void* gate, void* o, int B, int H, int dk, int dv,
+                        int dtype, float eps, cudaStream_t st) {
   if (dtype == RET_BF16)
-    return launch_step_t<__nv_bfloat16>(q, k, v, gammas, state, o, B, H, dk, dv, eps, st);
-  return launch_step_t<float>(q, k, v, gammas, state, o, B, H, dk, dv, eps, st);
+    return launch_step_t<__nv_bfloat16>(q, k, v, gammas, state, gate, o, B, H, dk, dv, eps, st);
+  return launch_step_t<float>(q, k, v, gammas, state, gate, o, B, H, dk, dv, eps, st);
 }
 
 }  // namespace ret

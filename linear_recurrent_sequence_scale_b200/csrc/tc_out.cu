@@ -72,6 +72,7 @@ template <bool GN> constexpr int threads() { return (6 + epi_warps<GN>()) * 32; 
 
 struct Params {
   const float* gammas;
+  const __nv_bfloat16* gate;  // null: no output gate
   __nv_bfloat16* o;
   int H, N, chunk, tpc, nc, dk, dv, dvs, nslices, ntiles;
   int chunked;     // 1: chunkwise form (R from the workspace), 0: parallel form
@@ -183,11 +184,12 @@ __device__ __forceinline__ float tree_sumsq32(const float (&x)[32]) {
   return t[0];
 }
 
-template <bool GN, int NQB, int KQ>
+template <bool GN, int NQB, int KQ, bool GATE>
 __global__ void __launch_bounds__(threads<GN>(), 1)
 chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_r,
-             const __grid_constant__ CUtensorMap tm_o, const Params p) {
+             const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_g,
+             const Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uintptr_t raw = reinterpret_cast<uintptr_t>(smem_raw);
   const uintptr_t aligned = (raw + 1023) & ~static_cast<uintptr_t>(1023);
@@ -297,6 +299,9 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       for (int tile = tile_at(p, k); tile >= 0 && ok; tile = tile_at(p, ++k)) {
         const Tile x = decode_tile(p, tile);
         while (ok && qn <= k) ok = issue_q(true);  // this tile's own Q
+        if (GATE) {  // the epilogue reads the gate tile about one tile later: into L2 now
+          for (int b = 0; b < vb; ++b) tma_prefetch_l2_3d(&tm_g, c0 + b * 64, x.n0, x.bh);
+        }
         for (int t = 0; t <= x.nt && ok; ++t) {
           if (t < x.nt) {
             const int key0 = x.cs + t * BN;
@@ -638,6 +643,48 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           }
         }
       }
+      if (GATE) {
+        // Output gate: y <- y swish(g) over the staged tile.  Each thread
+        // keeps 8 or 16 gate loads of 16 bytes in flight (the loader prefetched
+        // the tile into L2); a warp covers consecutive 16-byte pieces of one
+        // row, so the loads are coalesced and a quarter warp hits eight
+        // distinct 16-byte positions of a staged row.
+        ok = epi_bar_and<EPI>(xok);
+        const int cpr = p.dvs / 8;          // 16-byte pieces per row of the slice
+        const int et = threadIdx.x - 6 * 32;
+        const int pc = et % cpr;            // this thread's piece of every row it visits
+        const int rstep = EPI * 32 / cpr;   // rows visited together
+        const int nvis = BM / rstep;        // rows per thread
+        const __nv_bfloat16* gbase =
+            p.gate + ((size_t)x.bh * p.N + x.n0) * p.dv + c0 + pc * 8;
+        const uint32_t sbase = stage_a + (pc >> 3) * QBOX;
+        constexpr int GB = GN ? 8 : 16;     // gate loads in flight per thread (registers)
+        for (int v0 = 0; v0 < nvis; v0 += GB) {
+          uint4 gv[GB];
+#pragma unroll
+          for (int j = 0; j < GB; ++j) {
+            const int row = et / cpr + (v0 + j) * rstep;
+            if (v0 + j < nvis && x.n0 + row < p.N)
+              gv[j] = __ldg(reinterpret_cast<const uint4*>(gbase + (size_t)row * p.dv));
+          }
+#pragma unroll
+          for (int j = 0; j < GB; ++j) {
+            const int row = et / cpr + (v0 + j) * rstep;
+            if (v0 + j >= nvis || x.n0 + row >= p.N) continue;
+            const uint32_t a = sbase + row * 128 + (((pc & 7) ^ (row & 7)) * 16);
+            const uint4 yv = ld_shared_v4(a);
+            const uint32_t yi[4] = {yv.x, yv.y, yv.z, yv.w};
+            const uint32_t gi[4] = {gv[j].x, gv[j].y, gv[j].z, gv[j].w};
+            uint32_t r[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              r[e] = pack_bf16(bf16lo_to_f32(yi[e]) * swishf(bf16lo_to_f32(gi[e])),
+                               bf16hi_to_f32(yi[e]) * swishf(bf16hi_to_f32(gi[e])));
+            st_shared_v4(a, r[0], r[1], r[2], r[3]);
+          }
+        }
+        xok = ok;
+      }
       fence_proxy_async_smem();
       ok = epi_bar_and<EPI>(xok);
       if (warp == 6 && lane == 0) {
@@ -664,12 +711,14 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 int tc_out_device_error() { return read_clear_device_error(); }
 
 cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const float* gammas,
-                          int chunk, const void* ws, int has_state0, void* o, int B, int H, int N,
-                          int dk, int dv, float eps, int parallel_form, cudaStream_t st) {
+                          int chunk, const void* ws, int has_state0, const void* gate, void* o,
+                          int B, int H, int N, int dk, int dv, float eps, int parallel_form,
+                          cudaStream_t st) {
   using namespace k3;
   const uint64_t BH = (uint64_t)B * H;
   Params p;
   p.gammas = gammas;
+  p.gate = static_cast<const __nv_bfloat16*>(gate);
   p.o = static_cast<__nv_bfloat16*>(o);
   p.H = H;
   p.N = N;
@@ -698,10 +747,16 @@ cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const flo
   if (nclusters < 1) nclusters = 1;
   p.grouped = p.tpc > 1 && ntiles / p.tpc >= 4 * nclusters;
 
-  CUtensorMap tm_q, tm_k, tm_v, tm_r, tm_o;
+  CUtensorMap tm_q, tm_k, tm_v, tm_r, tm_o, tm_g;
   if ((e = make_tmap_bf16_3d(&tm_q, q, dk, N, BH, 64, BM)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_3d(&tm_k, k, dk, N, BH, 64, BN)) != cudaSuccess) return e;
   if ((e = make_tmap_bf16_3d(&tm_o, o, dv, N, BH, 64, BM)) != cudaSuccess) return e;
+  if (gate) {
+    if ((e = make_tmap_bf16_3d(&tm_g, const_cast<void*>(gate), dv, N, BH, 64, BM)) != cudaSuccess)
+      return e;
+  } else {
+    tm_g = tm_o;  // never read
+  }
   if ((e = make_tmap_bf16_3d(&tm_v, v, dv, N, BH, 64, 64)) != cudaSuccess) return e;
   if (ws) {
     if ((e = make_tmap_bf16_3d(&tm_r, ws, dv, dk, BH * p.nc, 64, 64)) != cudaSuccess) return e;
@@ -740,20 +795,25 @@ cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const flo
       if (max_clusters < 1) return cudaErrorInvalidConfiguration;
       if (cfg.gridDim.y > static_cast<unsigned>(max_clusters)) cfg.gridDim.y = max_clusters;
     }
-    return cudaLaunchKernelEx(&cfg, fn, tm_q, tm_k, tm_v, tm_r, tm_o, p);
+    return cudaLaunchKernelEx(&cfg, fn, tm_q, tm_k, tm_v, tm_r, tm_o, tm_g, p);
   };
-  auto by_dk = [&](auto gn, auto q) -> cudaError_t {
+  auto by_dk = [&](auto gn, auto q, auto gt) -> cudaError_t {
     constexpr bool G = decltype(gn)::value;
     constexpr int QB = decltype(q)::value;
-    if (dk == 64) return launch(chunk_out_tc<G, QB, 1>);
-    if (dk == 128) return launch(chunk_out_tc<G, QB, 2>);
-    return launch(chunk_out_tc<G, QB, 4>);
+    constexpr bool GT = decltype(gt)::value;
+    if (dk == 64) return launch(chunk_out_tc<G, QB, 1, GT>);
+    if (dk == 128) return launch(chunk_out_tc<G, QB, 2, GT>);
+    return launch(chunk_out_tc<G, QB, 4, GT>);
   };
   using T1 = std::integral_constant<int, 1>;
   using T2 = std::integral_constant<int, 2>;
-  if (eps >= 0.f)
-    return nqb == 1 ? by_dk(std::true_type{}, T1{}) : by_dk(std::true_type{}, T2{});
-  return nqb == 1 ? by_dk(std::false_type{}, T1{}) : by_dk(std::false_type{}, T2{});
+  auto by_q = [&](auto gn, auto gt) -> cudaError_t {
+    return nqb == 1 ? by_dk(gn, T1{}, gt) : by_dk(gn, T2{}, gt);
+  };
+  auto by_gn = [&](auto gt) -> cudaError_t {
+    return eps >= 0.f ? by_q(std::true_type{}, gt) : by_q(std::false_type{}, gt);
+  };
+  return gate ? by_gn(std::true_type{}) : by_gn(std::false_type{});
 }
 
 }  // namespace ret

@@ -141,3 +141,27 @@ def test_chunkwise_phases_reject_bad_arguments(lib):
     # state to copy
     assert output(N=0, q=None, k=None, v=None, o=None, ws=None, wsb=0) == ret.RET_OK
     assert states(N=0, k=None, v=None, ws=None, wsb=0) == ret.RET_OK
+
+
+def test_gated_entry_points_reject_bad_arguments(lib):
+    """The gate is checked like the other operands (16-byte alignment); a
+    NULL gate is the ungated call, so the ungated argument errors still show."""
+    need = lib.ret_chunkwise_workspace(1, 2, 300, 64, 64, 64, 0)
+    par = lambda g=A, o=A, N=16, eps=-1.0: lib.ret_parallel_gated(
+        A, A, A, A, g, o, 1, 2, N, 64, 64, 1, eps, None)
+    chk = lambda g=A, ws=A, N=300: lib.ret_chunkwise_gated(
+        A, A, A, A, 64, None, None, g, A, 1, 2, N, 64, 64, 0, -1.0, ws, need, None)
+    out = lambda g=A, eps=-1.0: lib.ret_chunkwise_output_gated(
+        A, A, A, A, 64, 0, g, A, 1, 2, 300, 64, 64, 0, eps, A, need, None)
+    stp = lambda g=A, s=A: lib.ret_step_gated(A, A, A, A, s, g, A, 2, 2, 64, 64, 1, -1.0, None)
+    assert par(g=M) == ret.RET_EINVAL
+    assert par(o=None) == ret.RET_EINVAL
+    assert par(eps=float("nan")) == ret.RET_EINVAL
+    assert par(N=0, g=None, o=None) == ret.RET_OK
+    assert chk(g=M) == ret.RET_EINVAL
+    assert chk(ws=None) == ret.RET_EWORKSPACE
+    assert chk(N=0, g=None) == ret.RET_OK
+    assert out(g=M) == ret.RET_EINVAL
+    assert out(eps=float("nan")) == ret.RET_EINVAL
+    assert stp(g=M) == ret.RET_EINVAL
+    assert stp(s=None) == ret.RET_EINVAL

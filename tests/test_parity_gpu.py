@@ -155,6 +155,24 @@ def test_chunkwise_in_two_phases(torch_cuda, ret, dt, chunk, gn):
     assert torch.equal(o, o1) and torch.equal(s, s1)
 
 
+@pytest.mark.parametrize("gn", [None, 1e-5])
+def test_chunkwise_strong_and_weak_decays(torch_cuda, ret, gn):
+    """Decays on both sides of gamma^chunk = 2^-64: the kernel folds xi into
+    the mask and the epilogue for the weak ones and rescales Q for the strong
+    ones (0.5^256 and 0); both must match the oracle, with a state entering."""
+    torch = torch_cuda
+    B, H, N, dk, dv, C = 1, 4, 700, 128, 256, 256
+    gam = [0.5, 0.9, 0.999, 0.0]
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=43, with_state=True, gammas=gam)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    o, s = ret.chunkwise(q, k, v, g, C, state_in=_dev(inp["state"]), return_state=True, gn_eps=gn)
+    torch.cuda.synchronize()
+    o_ref, s_ref = _ref_chunkwise(inp, C, gn, True)
+    assert _rel(o, o_ref) <= TOL["bf16"]
+    assert _rel(s, s_ref) <= STATE_TOL
+
+
 def test_groupnorm_far_from_zero_mean(torch_cuda, ret):
     """GroupNorm where every output row carries a large common offset and the
     32-column groups differ in spread by 30x: the normalised deviations must
@@ -177,6 +195,76 @@ def test_groupnorm_far_from_zero_mean(torch_cuda, ret):
     torch.cuda.synchronize()
     assert _rel(o, o_ref) <= TOL["bf16"]
     assert _rel(op, p_ref) <= TOL["bf16"]
+
+
+# --- gated output: swish(G) (.) Y -----------------------------------------------
+
+GATED_CASES = [
+    # form, dtype, B, H, N, dk, dv, chunk, gn_eps
+    ("chunkwise", "bf16", 1, 2, 1000, 256, 512, 512, 1e-5),   # tensor cores, 2 d_v slices
+    ("chunkwise", "bf16", 2, 2, 333, 128, 128, 128, None),    # tensor cores, ragged tail
+    ("parallel", "bf16", 1, 3, 300, 64, 256, None, 1e-5),
+    ("chunkwise", "f32", 1, 2, 200, 64, 96, 64, 1e-5),        # SIMT path
+    ("parallel", "f32", 1, 2, 130, 32, 40, None, None),
+]
+
+
+@pytest.mark.parametrize("case", GATED_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_gated_output_parity(torch_cuda, ret, case):
+    torch = torch_cuda
+    form, dt, B, H, N, dk, dv, chunk, gn = case
+    inp = wl.make_inputs(B, H, N, dk, dv, dt, seed=51 + N, with_state=True)
+    rng = np.random.default_rng(52 + N)
+    gate = wl.from_values(rng.standard_normal((B, H, N, dv)) * 2.0, dt)
+    q, k, v, gd = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"]), _dev(gate)
+    g = _gam(torch, inp["gammas"])
+    if form == "chunkwise":
+        o, s = ret.chunkwise(q, k, v, g, chunk, state_in=_dev(inp["state"]), return_state=True,
+                             gn_eps=gn, gate=gd)
+        y_ref, s_ref = _ref_chunkwise(inp, chunk, gn, True)
+    else:
+        o = ret.parallel(q, k, v, g, gn_eps=gn, gate=gd)
+        y_ref, _ = oracle.parallel(inp["q"].exact, inp["k"].exact, inp["v"].exact, inp["gammas"])
+        if gn is not None:
+            y_ref = oracle.group_norm(y_ref, gn)
+    torch.cuda.synchronize()
+    assert _rel(o, oracle.gated(y_ref, gate.exact)) <= TOL[dt]
+    if form == "chunkwise":
+        assert _rel(s, s_ref) <= STATE_TOL
+
+
+@pytest.mark.parametrize("gn", [None, 1e-5])
+def test_gated_step_parity(torch_cuda, ret, gn):
+    torch = torch_cuda
+    B, H, dk, dv = 2, 3, 64, 256
+    inp = wl.make_inputs(B, H, 1, dk, dv, "bf16", seed=61, with_state=True)
+    gate = wl.from_values(np.random.default_rng(62).standard_normal((B, H, dv)), "bf16")
+    state = _dev(inp["state"])
+    o = ret.step(_dev(inp["q"])[:, :, 0].contiguous(), _dev(inp["k"])[:, :, 0].contiguous(),
+                 _dev(inp["v"])[:, :, 0].contiguous(), _gam(torch, inp["gammas"]), state,
+                 gn_eps=gn, gate=_dev(gate))
+    torch.cuda.synchronize()
+    y_ref, s_ref = oracle.step(inp["q"].exact[:, :, 0], inp["k"].exact[:, :, 0],
+                               inp["v"].exact[:, :, 0], inp["gammas"], inp["state"].exact)
+    if gn is not None:
+        y_ref = oracle.group_norm(y_ref, gn)
+    assert _rel(o, oracle.gated(y_ref, gate.exact)) <= TOL["bf16"]
+    assert _rel(state, s_ref) <= STATE_TOL
+
+
+def test_gate_none_is_the_ungated_call(torch_cuda, ret):
+    """gate=None runs the ungated entry point; a gate of +40 (swish(40) = 40
+    in bf16 arithmetic) scales the ungated result by 40."""
+    torch = torch_cuda
+    B, H, N, dk, dv, C = 1, 2, 300, 128, 256, 128
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=71)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    o0 = ret.chunkwise(q, k, v, g, C, gn_eps=1e-5)
+    o1 = ret.chunkwise(q, k, v, g, C, gn_eps=1e-5,
+                       gate=torch.full_like(o0, 40.0))
+    torch.cuda.synchronize()
+    assert _rel(o1, 40.0 * wl.from_torch(o0)) <= 1e-2
 
 
 # --- parallel form -----------------------------------------------------------------
