@@ -204,6 +204,27 @@ RET_API int ret_step_gated(const void* q, const void* k, const void* v, const fl
                    float* state, const void* gate, void* o, int B, int H, int dk, int dv,
                    int dtype, float gn_eps, void* stream);
 
+/*
+ * State entering span r of a sequence split into spans held by different GPUs
+ * (sequence parallelism for the chunkwise form).  The carried state obeys
+ * the chunk recurrence ("RetNet - Retentive Network - A Successor to
+ * Transformer for LLMs", Key Equations, Chunkwise Recurrent) at span
+ * granularity: with S_local(g) the end state of span g computed from a zero
+ * state (ret_chunkwise_states with state_in = NULL) and N_g its length,
+ *     state_in = gamma^(N_0+...+N_(r-1)) state0
+ *              + sum_{g<r} gamma^(N_(g+1)+...+N_(r-1)) S_local(g).
+ *   locals   : device, [r][B][H][dk][dv] float32 (the gathered end states of
+ *              spans 0 .. r-1; may be NULL when r == 0).
+ *   spans    : HOST array of r span lengths (tokens, >= 0).
+ *   state0   : device [B][H][dk][dv] float32 entering span 0, or NULL (zero).
+ *   state_in : device [B][H][dk][dv] float32, written.  r == number of spans
+ *              gives the end state of the whole sequence.
+ * Supported: r <= 64.  All device pointers 16-byte aligned.
+ */
+RET_API int ret_state_combine(const float* locals, const int* spans, int r, const float* gammas,
+                      const float* state0, float* state_in, int B, int H, int dk, int dv,
+                      void* stream);
+
 /* Human-readable name of a ret_status value (static storage). */
 RET_API const char* ret_status_string(int status);
 

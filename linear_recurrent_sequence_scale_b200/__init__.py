@@ -38,6 +38,7 @@ SIGNATURES = {
     "ret_chunkwise_output_gated": (_I, [_P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I,
                                         _F, _P, _S, _P]),
     "ret_step_gated": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "ret_state_combine": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
     "ret_status_string": (ctypes.c_char_p, [_I]),
     "ret_last_cuda_error": (_I, []),
     "ret_version": (ctypes.c_char_p, []),
@@ -274,6 +275,31 @@ def chunkwise_output(q, k, v, gammas, chunk, workspace, has_state_in=False, gn_e
                                            _ptr(workspace), ws_bytes, _stream(dev))
     if s != RET_OK:
         _raise("ret_chunkwise_output", s)
+    return out
+
+
+def state_combine(locals_, spans, r, gammas, state0=None, out=None):
+    """State entering span r of a sequence split into spans (ret_state_combine).
+    locals_: [R,B,H,dk,dv] float32 end states of the spans computed from a zero
+    state; spans: R span lengths (host ints); state0: state entering span 0 or
+    None.  r = R gives the end state of the whole sequence."""
+    torch = _torch()
+    R, B, H, dk, dv = locals_.shape
+    dev = locals_.device
+    _check(locals_, "locals", dtype=torch.float32, device=dev)
+    if not 0 <= r <= R or len(spans) != R:
+        raise ValueError("need 0 <= r <= number of spans and one length per span")
+    _check(gammas, "gammas", dtype=torch.float32, shape=(H,), device=dev)
+    if state0 is not None:
+        _check(state0, "state0", dtype=torch.float32, shape=(B, H, dk, dv), device=dev)
+    if out is None:
+        out = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    _check(out, "out", dtype=torch.float32, shape=(B, H, dk, dv), device=dev)
+    sp = (ctypes.c_int * max(R, 1))(*[int(n) for n in spans])
+    s = load_library().ret_state_combine(_ptr(locals_), sp, int(r), _ptr(gammas), _ptr(state0),
+                                         _ptr(out), B, H, dk, dv, _stream(dev))
+    if s != RET_OK:
+        _raise("ret_state_combine", s)
     return out
 
 

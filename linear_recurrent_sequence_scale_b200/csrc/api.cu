@@ -223,6 +223,21 @@ int ret_chunkwise(const void* q, const void* k, const void* v, const float* gamm
                              dv, dtype, gn_eps, workspace, workspace_bytes, stream);
 }
 
+int ret_state_combine(const float* locals, const int* spans, int r, const float* gammas,
+                      const float* state0, float* state_in, int B, int H, int dk, int dv,
+                      void* stream) {
+  if (B < 1 || H < 1 || dk < 8 || dv < 8 || dk % 8 || dv % 8) return RET_EINVAL;
+  if (r < 0 || (r > 0 && (!locals || !spans)) || !gammas || !state_in) return RET_EINVAL;
+  if (r > ret::kMaxSpans) return RET_EUNSUPPORTED;
+  if ((int64_t)B * H * dk * dv > ((int64_t)1 << 40)) return RET_EUNSUPPORTED;
+  for (int g = 0; g < r; ++g)
+    if (spans[g] < 0) return RET_EINVAL;
+  if ((locals && !aligned16(locals)) || (state0 && !aligned16(state0)) || !aligned16(state_in))
+    return RET_EINVAL;
+  return cuda_status(ret::launch_state_combine(locals, spans, r, gammas, state0, state_in, B, H,
+                                               dk, dv, static_cast<cudaStream_t>(stream)));
+}
+
 int ret_step_gated(const void* q, const void* k, const void* v, const float* gammas,
                    float* state, const void* gate, void* o, int B, int H, int dk, int dv,
                    int dtype, float gn_eps, void* stream) {

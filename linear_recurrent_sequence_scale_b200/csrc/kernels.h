@@ -22,6 +22,12 @@ cudaError_t launch_simt_output(const void* q, const void* k, const void* v, cons
                                int chunk, const void* gate, void* o, int B, int H, int N, int dk,
                                int dv, int dtype, float eps, const void* ws, cudaStream_t st);
 
+// State entering span r of a sequence split across GPUs (seqpar.cu).
+constexpr int kMaxSpans = 64;
+cudaError_t launch_state_combine(const float* locals, const int* spans, int r,
+                                 const float* gammas, const float* state0, float* out, int B,
+                                 int H, int dk, int dv, cudaStream_t st);
+
 cudaError_t launch_simt_parallel(const void* q, const void* k, const void* v, const float* gammas,
                                  const void* gate, void* o, int B, int H, int N, int dk, int dv,
                                  int dtype, float eps, cudaStream_t st);

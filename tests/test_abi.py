@@ -165,3 +165,19 @@ def test_gated_entry_points_reject_bad_arguments(lib):
     assert out(eps=float("nan")) == ret.RET_EINVAL
     assert stp(g=M) == ret.RET_EINVAL
     assert stp(s=None) == ret.RET_EINVAL
+
+
+def test_state_combine_rejects_bad_arguments(lib):
+    spans = (ctypes.c_int * 3)(5, 7, 9)
+    bad = (ctypes.c_int * 3)(5, -1, 9)
+    f = lambda loc=A, sp=spans, r=3, g=A, s0=None, out=A, dk=64: lib.ret_state_combine(
+        loc, sp, r, g, s0, out, 1, 2, dk, 64, None)
+    assert f(r=-1) == ret.RET_EINVAL
+    assert f(loc=None) == ret.RET_EINVAL
+    assert f(sp=None) == ret.RET_EINVAL
+    assert f(sp=bad) == ret.RET_EINVAL
+    assert f(out=None) == ret.RET_EINVAL
+    assert f(out=M) == ret.RET_EINVAL
+    assert f(s0=M) == ret.RET_EINVAL
+    assert f(dk=12) == ret.RET_EINVAL
+    assert f(r=65) == ret.RET_EUNSUPPORTED

@@ -267,6 +267,53 @@ def test_gate_none_is_the_ungated_call(torch_cuda, ret):
     assert _rel(o1, 40.0 * wl.from_torch(o0)) <= 1e-2
 
 
+# --- sequence parallelism: spans of one sequence, emulated on one GPU -------------
+
+def test_state_combine_matches_the_span_recurrence(torch_cuda, ret):
+    torch = torch_cuda
+    rng = np.random.default_rng(91)
+    R, B, H, dk, dv = 4, 2, 3, 64, 128
+    loc = rng.standard_normal((R, B, H, dk, dv)).astype(np.float32)
+    s0 = rng.standard_normal((B, H, dk, dv)).astype(np.float32)
+    gam = np.array([0.9, 0.999, 0.5], dtype=np.float32)
+    spans = [100, 0, 37, 512]
+    for r in range(R + 1):
+        ref = s0.astype(np.float64)
+        for i in range(r):
+            ref = gam.astype(np.float64)[None, :, None, None] ** spans[i] * ref + loc[i]
+        got = ret.state_combine(torch.from_numpy(loc).cuda(), spans, r,
+                                torch.from_numpy(gam).cuda(), torch.from_numpy(s0).cuda())
+        torch.cuda.synchronize()
+        assert _rel(got, ref) <= 1e-6
+
+
+def test_sequence_parallel_spans_on_one_gpu(torch_cuda, ret):
+    """Three ranks' spans run one after another on this GPU with the real
+    kernels (the all-gather replaced by stacking): each span's output and the
+    sequence's end state against the oracle over the unsplit sequence."""
+    from linear_recurrent_sequence_scale_b200 import seqpar
+    torch = torch_cuda
+    B, H, N, dk, dv, C = 1, 2, 1500, 128, 256, 256
+    spans = [700, 300, 500]
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=92, with_state=True)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    s0 = _dev(inp["state"])
+    cut = np.cumsum([0] + spans)
+    part = lambda x, r: x[:, :, cut[r]:cut[r + 1]].contiguous()
+    locs = torch.stack([seqpar.local_end_state(part(q, r), part(k, r), part(v, r), g, C)
+                        for r in range(3)])
+    outs = []
+    for r in range(3):
+        o, s = seqpar.span_output(part(q, r), part(k, r), part(v, r), g, C, locs, spans, r,
+                                  state0=s0, gn_eps=1e-5, return_state=True)
+        outs.append(o)
+    torch.cuda.synchronize()
+    o_ref, s_ref = _ref_chunkwise(inp, C, 1e-5, True)
+    assert _rel(torch.cat(outs, dim=2), o_ref) <= TOL["bf16"]
+    assert _rel(s, s_ref) <= STATE_TOL
+
+
 # --- parallel form -----------------------------------------------------------------
 
 PAR_CASES = [
