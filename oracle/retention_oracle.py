@@ -161,6 +161,43 @@ def group_norm(o, eps: float):
     return (o - mu) / np.sqrt(var + eps)
 
 
+def backward(q, k, v, gammas, d_o, state_in=None, d_state_out=None):
+    """Gradients of the retention outputs and the final state with respect to
+    q, k, v and the initial state: the adjoint of the forms above ([RetNet
+    blog] Key Equations; the pages call the parallel form the training form
+    and give no gradient, so this is the chain rule written out).  Per
+    (b, h), with A = Q K^T (.) D, xi_n = gamma^(n+1), z_m = gamma^(N-1-m),
+    O = A V + (Q (.) xi) S_in and S_out = K^T (V (.) z) + gamma^N S_in:
+        dA    = dO V^T (.) D
+        dQ    = dA K + xi (.) (dO S_in^T)
+        dK    = dA^T Q + z (.) (V dS_out^T)
+        dV    = A^T dO + z (.) (K dS_out)
+        dS_in = (Q (.) xi)^T dO + gamma^N dS_out.
+    Returns (dq, dk, dv, d_state_in)."""
+    q, k, v, d_o = _f64(q), _f64(k), _f64(v), _f64(d_o)
+    B, H, N, dk = q.shape
+    dv = v.shape[-1]
+    s_in = np.zeros((B, H, dk, dv)) if state_in is None else _f64(state_in)
+    d_s = np.zeros((B, H, dk, dv)) if d_state_out is None else _f64(d_state_out)
+    dq, dkk, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    ds_in = np.zeros((B, H, dk, dv))
+    n = np.arange(N)
+    for h in range(H):
+        g = float(gammas[h])
+        D = decay_mask(g, N)
+        xi = np.power(g, n + 1.0)
+        z = np.power(g, N - 1.0 - n)
+        for b in range(B):
+            Q, K, V, dO = q[b, h], k[b, h], v[b, h], d_o[b, h]
+            A = (Q @ K.T) * D
+            dA = (dO @ V.T) * D
+            dq[b, h] = dA @ K + xi[:, None] * (dO @ s_in[b, h].T)
+            dkk[b, h] = dA.T @ Q + z[:, None] * (V @ d_s[b, h].T)
+            dvv[b, h] = A.T @ dO + z[:, None] * (K @ d_s[b, h])
+            ds_in[b, h] = (Q * xi[:, None]).T @ dO + g ** N * d_s[b, h]
+    return dq, dkk, dvv, ds_in
+
+
 def swish(x):
     """swish(x) = x * sigmoid(x) = x / (1 + exp(-x)), the gate activation of
     the retention block ([RetNet blog] core components, item 4: GroupNorm

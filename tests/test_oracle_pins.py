@@ -249,6 +249,61 @@ def test_msr_gammas_exact():
     assert np.all((g > 0) & (g < 1))
 
 
+# --- backward: the chain rule against finite differences ----------------------
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_backward_matches_finite_differences(with_state):
+    """Directional derivatives of L = <dO, O> + <dS, S_out> (O, S_out from the
+    parallel form with the closed-form state) by central differences, against
+    <gradient, direction> from oracle.backward; also through the chunkwise
+    form, whose agreement with the parallel form is pinned above."""
+    rng = np.random.default_rng(31)
+    B, H, N, dk, dv = 1, 2, 9, 3, 4
+    q, k, v, s0 = _rand(rng, B, H, N, dk, dv, state=True)
+    s0 = s0 if with_state else None
+    gam = [0.8, 0.5]
+    dO = rng.standard_normal((B, H, N, dv))
+    dS = rng.standard_normal((B, H, dk, dv))
+    gq, gk, gv, gs = oracle.backward(q, k, v, gam, dO, s0, dS)
+
+    def loss(q_, k_, v_, s_, form):
+        if form == "parallel":
+            o, s = oracle.parallel(q_, k_, v_, gam, s_)
+        else:
+            o, s = oracle.chunkwise(q_, k_, v_, gam, 4, s_)
+        return float((dO * o).sum() + (dS * s).sum())
+
+    eps = 1e-6
+    for form in ("parallel", "chunkwise"):
+        for which in range(4 if with_state else 3):
+            U = [np.zeros_like(q), np.zeros_like(k), np.zeros_like(v),
+                 np.zeros((B, H, dk, dv))]
+            U[which] = rng.standard_normal(U[which].shape)
+            args_p = [q + eps * U[0], k + eps * U[1], v + eps * U[2]]
+            args_m = [q - eps * U[0], k - eps * U[1], v - eps * U[2]]
+            sp = None if s0 is None else s0 + eps * U[3]
+            sm = None if s0 is None else s0 - eps * U[3]
+            fd = (loss(*args_p, sp, form) - loss(*args_m, sm, form)) / (2 * eps)
+            an = float((gq * U[0]).sum() + (gk * U[1]).sum() + (gv * U[2]).sum()
+                       + (gs * U[3]).sum())
+            assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (form, which, fd, an)
+
+
+def test_backward_gamma_zero_and_one():
+    """gamma = 0: O_n = (q_n . k_n) v_n, so dq_n = (dO_n . v_n) k_n; gamma = 1
+    with dS = 0: dV_m = sum over n >= m of (q_n . k_m) dO_n (causal sums)."""
+    rng = np.random.default_rng(32)
+    q, k, v, _ = _rand(rng, 1, 1, 6, 3, 2, state=False)
+    dO = rng.standard_normal((1, 1, 6, 2))
+    gq, _, _, _ = oracle.backward(q, k, v, [0.0], dO)
+    exp_q = np.einsum("nj,nj->n", dO[0, 0], v[0, 0])[:, None] * k[0, 0]
+    np.testing.assert_allclose(gq[0, 0], exp_q, rtol=1e-12, atol=1e-12)
+    _, _, gv, _ = oracle.backward(q, k, v, [1.0], dO)
+    exp_v = np.stack([sum((q[0, 0, n] @ k[0, 0, m]) * dO[0, 0, n] for n in range(m, 6))
+                      for m in range(6)])
+    np.testing.assert_allclose(gv[0, 0], exp_v, rtol=1e-12, atol=1e-12)
+
+
 # --- gate: swish(G) (.) Y ------------------------------------------------------
 
 def test_swish_identities():
