@@ -23,6 +23,7 @@ is needed between steps.  The same line carries:
   parallel      the parallel form on the 1.3B-class layer (8 x 8 heads x 2048)
   long_64k      chunkwise over 65536 tokens (1 x 16 heads)
   gated         the headline step with the output gate swish(G) (.) GN(o)
+  backward      the chunkwise backward on the 1.3B-class layer
   cpu_baseline  the float64 CPU oracle on a bounded sample of the same
                 workload (rank 0, N = 1 only)
 With N > 1 (torchrun) every rank runs the same per-GPU step on its own GPU
@@ -568,6 +569,25 @@ def run_ours(args):
                              "ms": cl * 1e3, "tflops": Fl / cl / 1e12,
                              "frac_tc": Fl / cl / 1e12 / peak}
         del ql, kl, vl, ol, sl, wsl
+        torch.cuda.empty_cache()
+
+        # ---------------- backward on the 1.3B-class layer ----------------
+        wb = wl.WORKLOADS["l1p3b_bf16"]
+        qb, kb, vb, gb = make_qkv(torch, wb.B, wb.H, wb.N, wb.dk, wb.dv, device, seed=7000 + rank)
+        dob = (torch.randn(vb.shape, device=device) * 0.1).bfloat16()
+        wsb = torch.empty(ret.load_library().ret_chunkwise_backward_workspace(
+            wb.B, wb.H, wb.N, wb.dk, wb.dv, wb.chunk, ret.RET_BF16), dtype=torch.uint8,
+            device=device)
+        tb, _ = timed(lambda: ret.chunkwise_backward(qb, kb, vb, gb, wb.chunk, dob, workspace=wsb),
+                      3, 1, stream, device)
+        launches += 3 * 3
+        Fb = 2 * chunkwise_flops(wb.B, wb.H, wb.N, wb.dk, wb.dv, wb.chunk)
+        cb = tb / 3
+        extra["backward"] = {"workload": "l1p3b_bf16 chunkwise backward (dq, dk, dv)",
+                             "ms": cb * 1e3, "tokens_per_s": wb.B * wb.N / cb,
+                             "tflops": Fb / cb / 1e12,
+                             "note": "CUDA cores, float32; flops counted as twice the forward's"}
+        del qb, kb, vb, dob, wsb
         torch.cuda.empty_cache()
 
         # ---------------- gated output on the headline workload ----------------

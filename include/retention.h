@@ -225,6 +225,30 @@ RET_API int ret_state_combine(const float* locals, const int* spans, int r, cons
                       const float* state0, float* state_in, int B, int H, int dk, int dv,
                       void* stream);
 
+/*
+ * Backward of the chunkwise form (the training role; "RetNet - Retentive
+ * Network - A Successor to Transformer for LLMs", Key Equations: the pages
+ * give the forms, this is their chain rule): given dO, the gradient of the
+ * outputs o of ret_chunkwise without GroupNorm or gate, and d_state_out, that
+ * of its final state, it writes
+ *   grad_q, grad_k, grad_v : [B][H][N][dk|dv], dtype of the inputs (written)
+ *   d_state_in   : [B][H][dk][dv] float32, the gradient of state_in (or NULL)
+ *   state_in     : the forward call's initial state, or NULL (zero)
+ *   d_state_out  : [B][H][dk][dv] float32, or NULL (zero)
+ *   workspace    : at least ret_chunkwise_backward_workspace() bytes; holds
+ *                  the forward and the gradient chunk states in float32.
+ * Runs on the CUDA cores in float32 for either dtype and any chunk >= 1,
+ * dk, dv in [8, 512].  Errors as for ret_chunkwise.
+ */
+RET_API size_t ret_chunkwise_backward_workspace(int B, int H, int N, int dk, int dv, int chunk,
+                                        int dtype);
+RET_API int ret_chunkwise_backward(const void* q, const void* k, const void* v,
+                           const float* gammas, int chunk, const float* state_in,
+                           const void* d_o, const float* d_state_out, void* grad_q,
+                           void* grad_k, void* grad_v, float* d_state_in, int B, int H, int N,
+                           int dk, int dv, int dtype, void* workspace, size_t workspace_bytes,
+                           void* stream);
+
 /* Human-readable name of a ret_status value (static storage). */
 RET_API const char* ret_status_string(int status);
 

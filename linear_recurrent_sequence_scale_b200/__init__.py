@@ -39,6 +39,9 @@ SIGNATURES = {
                                         _F, _P, _S, _P]),
     "ret_step_gated": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
     "ret_state_combine": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "ret_chunkwise_backward_workspace": (_S, [_I, _I, _I, _I, _I, _I, _I]),
+    "ret_chunkwise_backward": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I,
+                                    _I, _I, _I, _P, _S, _P]),
     "ret_status_string": (ctypes.c_char_p, [_I]),
     "ret_last_cuda_error": (_I, []),
     "ret_version": (ctypes.c_char_p, []),
@@ -276,6 +279,34 @@ def chunkwise_output(q, k, v, gammas, chunk, workspace, has_state_in=False, gn_e
     if s != RET_OK:
         _raise("ret_chunkwise_output", s)
     return out
+
+
+def chunkwise_backward(q, k, v, gammas, chunk, d_o, state_in=None, d_state_out=None,
+                       workspace=None):
+    """Gradients of ret_chunkwise (no GroupNorm, no gate): returns
+    (dq, dk, dv, d_state_in) for the output gradient d_o [B,H,N,dv] and the
+    optional final-state gradient d_state_out (ret_chunkwise_backward)."""
+    torch = _torch()
+    B, H, N, dk, dv, dev = _seq_args(q, k, v, gammas)
+    _check(d_o, "d_o", dtype=q.dtype, shape=(B, H, N, dv), device=dev)
+    sshape = (B, H, dk, dv)
+    for t, name in ((state_in, "state_in"), (d_state_out, "d_state_out")):
+        if t is not None:
+            _check(t, name, dtype=torch.float32, shape=sshape, device=dev)
+    dq, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ds = torch.empty(sshape, dtype=torch.float32, device=dev)
+    lib = load_library()
+    need = int(lib.ret_chunkwise_backward_workspace(B, H, N, dk, dv, int(chunk), _dtype_code(q)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    s = lib.ret_chunkwise_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), int(chunk),
+                                   _ptr(state_in), _ptr(d_o), _ptr(d_state_out), _ptr(dq),
+                                   _ptr(dk_), _ptr(dv_), _ptr(ds), B, H, N, dk, dv,
+                                   _dtype_code(q), _ptr(workspace), wsb, _stream(dev))
+    if s != RET_OK:
+        _raise("ret_chunkwise_backward", s)
+    return dq, dk_, dv_, ds
 
 
 def state_combine(locals_, spans, r, gammas, state0=None, out=None):

@@ -223,6 +223,45 @@ int ret_chunkwise(const void* q, const void* k, const void* v, const float* gamm
                              dv, dtype, gn_eps, workspace, workspace_bytes, stream);
 }
 
+size_t ret_chunkwise_backward_workspace(int B, int H, int N, int dk, int dv, int chunk,
+                                        int dtype) {
+  if (check_seq_dims(B, H, N, dk, dv, dtype) != RET_OK || chunk < 1 || N == 0) return 0;
+  return ret::backward_workspace_bytes(B, H, N, dk, dv, chunk);
+}
+
+int ret_chunkwise_backward(const void* q, const void* k, const void* v, const float* gammas,
+                           int chunk, const float* state_in, const void* d_o,
+                           const float* d_state_out, void* dq, void* dk_, void* dv_,
+                           float* d_state_in, int B, int H, int N, int dk, int dv, int dtype,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  int s = check_seq_dims(B, H, N, dk, dv, dtype);
+  if (s) return s;
+  if (chunk < 1 || !gammas) return RET_EINVAL;
+  if ((state_in && !aligned16(state_in)) || (d_state_out && !aligned16(d_state_out)) ||
+      (d_state_in && !aligned16(d_state_in)))
+    return RET_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t state_bytes = sizeof(float) * (size_t)B * H * dk * dv;
+  if (N == 0) {
+    // No tokens: the final state is the initial one, so their gradients are equal.
+    if (!d_state_in) return RET_OK;
+    if (d_state_out)
+      return cuda_status(cudaMemcpyAsync(d_state_in, d_state_out, state_bytes,
+                                         cudaMemcpyDeviceToDevice, st));
+    return cuda_status(cudaMemsetAsync(d_state_in, 0, state_bytes, st));
+  }
+  if (!q || !k || !v || !d_o || !dq || !dk_ || !dv_) return RET_EINVAL;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_o) || !aligned16(dq) ||
+      !aligned16(dk_) || !aligned16(dv_))
+    return RET_EINVAL;
+  const size_t need = ret::backward_workspace_bytes(B, H, N, dk, dv, chunk);
+  if (!workspace || workspace_bytes < need) return RET_EWORKSPACE;
+  if (!aligned16(workspace)) return RET_EINVAL;
+  return cuda_status(ret::launch_chunkwise_backward(q, k, v, gammas, chunk, state_in, d_o,
+                                                    d_state_out, dq, dk_, dv_, d_state_in, B, H,
+                                                    N, dk, dv, dtype, workspace, st));
+}
+
 int ret_state_combine(const float* locals, const int* spans, int r, const float* gammas,
                       const float* state0, float* state_in, int B, int H, int dk, int dv,
                       void* stream) {

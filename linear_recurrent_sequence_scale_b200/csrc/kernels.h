@@ -22,6 +22,16 @@ cudaError_t launch_simt_output(const void* q, const void* k, const void* v, cons
                                int chunk, const void* gate, void* o, int B, int H, int N, int dk,
                                int dv, int dtype, float eps, const void* ws, cudaStream_t st);
 
+// Chunkwise backward on the CUDA cores (backward.cu); ws holds the forward
+// and the gradient chunk states in float32.
+size_t backward_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk);
+cudaError_t launch_chunkwise_backward(const void* q, const void* k, const void* v,
+                                      const float* gammas, int chunk, const float* state_in,
+                                      const void* dout, const float* d_state_out, void* dq,
+                                      void* dk_, void* dv_, float* d_state_in, int B, int H,
+                                      int N, int dk, int dv, int dtype, void* ws,
+                                      cudaStream_t st);
+
 // State entering span r of a sequence split across GPUs (seqpar.cu).
 constexpr int kMaxSpans = 64;
 cudaError_t launch_state_combine(const float* locals, const int* spans, int r,

@@ -181,3 +181,24 @@ def test_state_combine_rejects_bad_arguments(lib):
     assert f(s0=M) == ret.RET_EINVAL
     assert f(dk=12) == ret.RET_EINVAL
     assert f(r=65) == ret.RET_EUNSUPPORTED
+
+
+def test_backward_rejects_bad_arguments(lib):
+    need = lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 64, 64, 0)
+    assert need > 0 and lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 64, 0, 0) == 0
+
+    def call(q=A, dO=A, gq=A, ds=A, si=None, dso=None, ws=A, wsb=None, N=300, chunk=64, dt=0):
+        wsb = need if wsb is None else wsb
+        return lib.ret_chunkwise_backward(q, A, A, A, chunk, si, dO, dso, gq, A, A, ds,
+                                          1, 2, N, 64, 64, dt, ws, wsb, None)
+
+    assert call(q=None) == ret.RET_EINVAL
+    assert call(dO=None) == ret.RET_EINVAL
+    assert call(gq=M) == ret.RET_EINVAL
+    assert call(si=M) == ret.RET_EINVAL
+    assert call(ds=M) == ret.RET_EINVAL
+    assert call(chunk=0) == ret.RET_EINVAL
+    assert call(dt=5) == ret.RET_EINVAL
+    assert call(ws=None) == ret.RET_EWORKSPACE
+    assert call(wsb=need - 1) == ret.RET_EWORKSPACE
+    assert call(N=0, q=None, dO=None, gq=None, ds=None, ws=None, wsb=0) == ret.RET_OK

@@ -314,6 +314,43 @@ def test_sequence_parallel_spans_on_one_gpu(torch_cuda, ret):
     assert _rel(s, s_ref) <= STATE_TOL
 
 
+# --- backward ----------------------------------------------------------------------
+
+BWD_CASES = [
+    # dtype, B, H, N, dk, dv, chunk, state_in, d_state_out
+    ("f32", 1, 2, 200, 64, 96, 64, True, True),
+    ("f32", 2, 1, 130, 32, 40, 37, False, True),
+    ("f32", 1, 3, 257, 128, 128, 128, True, False),
+    ("bf16", 1, 2, 700, 128, 256, 256, True, True),
+    ("bf16", 1, 2, 333, 256, 512, 512, False, False),
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_chunkwise_backward_parity(torch_cuda, ret, case):
+    torch = torch_cuda
+    dt, B, H, N, dk, dv, chunk, with_s0, with_ds = case
+    inp = wl.make_inputs(B, H, N, dk, dv, dt, seed=101 + N, with_state=True)
+    rng = np.random.default_rng(102 + N)
+    d_o = wl.from_values(rng.standard_normal((B, H, N, dv)) * 0.1, dt)
+    d_s = rng.standard_normal((B, H, dk, dv)).astype(np.float32) if with_ds else None
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    s0 = _dev(inp["state"]) if with_s0 else None
+    gq, gk, gv, gs = ret.chunkwise_backward(
+        q, k, v, g, chunk, _dev(d_o), state_in=s0,
+        d_state_out=torch.from_numpy(d_s).cuda() if with_ds else None)
+    torch.cuda.synchronize()
+    rq, rk, rv, rs = oracle.backward(inp["q"].exact, inp["k"].exact, inp["v"].exact,
+                                     inp["gammas"], d_o.exact,
+                                     inp["state"].exact if with_s0 else None, d_s)
+    tol = TOL[dt]
+    assert _rel(gq, rq) <= tol
+    assert _rel(gk, rk) <= tol
+    assert _rel(gv, rv) <= tol
+    assert _rel(gs, rs) <= (1e-5 if dt == "f32" else 1e-4)
+
+
 # --- parallel form -----------------------------------------------------------------
 
 PAR_CASES = [
