@@ -61,7 +61,7 @@ template <int NQB> struct Layout {
   static constexpr int RING = (DATA_BYTES - NQB * QBUF) / STAGE;
   static constexpr int RING_OFF = NQB * QBUF;
   static_assert(RING >= 2 && RING_OFF + RING * STAGE <= DATA_BYTES, "ring layout");
-  static_assert((2 * RING + 15) * 8 <= SMEM_BYTES - ALIGN_SLACK - BAR_OFF, "barrier area");
+  static_assert((2 * RING + 17) * 8 <= SMEM_BYTES - ALIGN_SLACK - BAR_OFF, "barrier area");
 };
 static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA");
 // Epilogue warps: with GroupNorm (two passes over O and an exchange) two per
@@ -158,6 +158,18 @@ __device__ __forceinline__ void chan_merge(float& n_a, float& mean_a, float& m2_
   n_a = n;
 }
 
+// y <- y swish(g) on eight bf16 values (four packed pairs), g read from the
+// staged gate piece at the same place.
+__device__ __forceinline__ void gate_in_place(uint32_t& y0, uint32_t& y1, uint32_t& y2,
+                                              uint32_t& y3, const uint4 g) {
+  uint32_t* y[4] = {&y0, &y1, &y2, &y3};
+  const uint32_t gi[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    *y[e] = pack_bf16(bf16lo_to_f32(*y[e]) * swishf(bf16lo_to_f32(gi[e])),
+                      bf16hi_to_f32(*y[e]) * swishf(bf16hi_to_f32(gi[e])));
+}
+
 // Sum of 32 values as a balanced tree: depth 5 instead of a 32-long chain.
 __device__ __forceinline__ float tree_sum32(const float (&x)[32]) {
   float t[16];
@@ -222,7 +234,8 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   uint64_t* o_free = q_full + 10;
   uint64_t* gn_bar = q_full + 11;     // [2]
   uint64_t* drain = q_full + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 14);
+  uint64_t* g_full = q_full + 14;     // [2] gate tile in the staging buffer (boxes >= 1, box 0)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_full + 16);
   float* gn_red = reinterpret_cast<float*>(smem + GN_OFF);
 
   const int warp = threadIdx.x >> 5;
@@ -244,6 +257,8 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     mbar_init(o_full, 1);
     mbar_init(o_free, EPI);
     mbar_init(drain, 1);
+    mbar_init(&g_full[0], 1);
+    mbar_init(&g_full[1], 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -299,9 +314,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       for (int tile = tile_at(p, k); tile >= 0 && ok; tile = tile_at(p, ++k)) {
         const Tile x = decode_tile(p, tile);
         while (ok && qn <= k) ok = issue_q(true);  // this tile's own Q
-        if (GATE) {  // the epilogue reads the gate tile about one tile later: into L2 now
-          for (int b = 0; b < vb; ++b) tma_prefetch_l2_3d(&tm_g, c0 + b * 64, x.n0, x.bh);
-        }
+
         for (int t = 0; t <= x.nt && ok; ++t) {
           if (t < x.nt) {
             const int key0 = x.cs + t * BN;
@@ -523,6 +536,20 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       const uint32_t stage_a = smem_u32(smem + Q_OFF + (k % NQB) * QBUF);
       if (!epi_bar_and<EPI>(mbar_wait(o_full, k & 1, 212))) break;
       tc_fence_after();
+      // Output gate: its tile goes by TMA into this tile's Q buffer (the MMAs
+      // that read Q are done), where the epilogue stages the output, and is
+      // applied in place as each staged 16-byte piece is written.  Box 0 is
+      // loaded only after the two halves' GroupNorm statistics, which pass
+      // through the buffer's first 2 KB, have been read.
+      const int nblk = p.dvs / 64;
+      const bool late0 = GN && NH == 2;
+      if (GATE && warp == 6 && lane == 0) {
+        const int b0 = late0 ? 1 : 0;
+        mbar_arrive_expect_tx(&g_full[0], (nblk - b0) * QBOX);
+        for (int b = b0; b < nblk; ++b)
+          tma_load_3d(smem + Q_OFF + (k % NQB) * QBUF + b * QBOX, &tm_g, &g_full[0], c0 + b * 64,
+                      x.n0, x.bh);
+      }
       bool xok = true;
       const uint32_t row_a = stage_a + i * 128;
       if (GN) {
@@ -578,7 +605,12 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           epi_bar2<EPI>();
           const float m_o = part[(2 * (half ^ 1)) * 128 + i];
           const float q_o = part[(2 * (half ^ 1) + 1) * 128 + i];
+          if (GATE) fence_proxy_async_smem();  // these accesses before box 0's TMA write
           epi_bar2<EPI>();
+          if (GATE && warp == 6 && lane == 0) {
+            mbar_arrive_expect_tx(&g_full[1], QBOX);
+            tma_load_3d(smem + Q_OFF + (k % NQB) * QBUF, &tm_g, &g_full[1], c0, x.n0, x.bh);
+          }
           // merged in the same order by both halves: identical statistics
           const float mb = half ? m_a : m_o, qb = half ? q_a : q_o;
           if (half) { m_a = m_o; q_a = q_o; }
@@ -597,6 +629,10 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
                           gn_red[slot * 256 + 128 + i]);
         }
         const float inv = 1.0f / sqrtf(q_a / static_cast<float>(p.dv) + p.eps);
+        if (GATE) {
+          if (!mbar_wait(&g_full[0], k & 1, 214)) xok = false;
+          if (late0 && !mbar_wait(&g_full[1], k & 1, 215)) xok = false;
+        }
 #pragma unroll
         for (int g = 0; g < GN_G; ++g) {
           if (g < ncg) {
@@ -612,6 +648,8 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               const int phys = (((cg & 1) * 4 + c) ^ (i & 7));
+              if (GATE) gate_in_place(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3],
+                                      ld_shared_v4(rowa + phys * 16));
               st_shared_v4(rowa + phys * 16, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2],
                            pk[4 * c + 3]);
             }
@@ -621,6 +659,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         // Stage bf16 O in this tile's Q buffer as [64-column block][128 rows]
         // [128 B] with the 128-byte swizzle, then write it with coalesced TMA
         // stores; rows past N are clipped by the tensor map.
+        if (GATE && !mbar_wait(&g_full[0], k & 1, 214)) xok = false;
         for (int g = 0; g < ncg; ++g) {
           const int cg = cg0 + g;
           uint32_t v[32];
@@ -639,51 +678,11 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const int phys = (((cg & 1) * 4 + c) ^ (i & 7));
+            if (GATE) gate_in_place(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3],
+                                    ld_shared_v4(rowa + phys * 16));
             st_shared_v4(rowa + phys * 16, pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
           }
         }
-      }
-      if (GATE) {
-        // Output gate: y <- y swish(g) over the staged tile.  Each thread
-        // keeps 8 or 16 gate loads of 16 bytes in flight (the loader prefetched
-        // the tile into L2); a warp covers consecutive 16-byte pieces of one
-        // row, so the loads are coalesced and a quarter warp hits eight
-        // distinct 16-byte positions of a staged row.
-        ok = epi_bar_and<EPI>(xok);
-        const int cpr = p.dvs / 8;          // 16-byte pieces per row of the slice
-        const int et = threadIdx.x - 6 * 32;
-        const int pc = et % cpr;            // this thread's piece of every row it visits
-        const int rstep = EPI * 32 / cpr;   // rows visited together
-        const int nvis = BM / rstep;        // rows per thread
-        const __nv_bfloat16* gbase =
-            p.gate + ((size_t)x.bh * p.N + x.n0) * p.dv + c0 + pc * 8;
-        const uint32_t sbase = stage_a + (pc >> 3) * QBOX;
-        constexpr int GB = GN ? 8 : 16;     // gate loads in flight per thread (registers)
-        for (int v0 = 0; v0 < nvis; v0 += GB) {
-          uint4 gv[GB];
-#pragma unroll
-          for (int j = 0; j < GB; ++j) {
-            const int row = et / cpr + (v0 + j) * rstep;
-            if (v0 + j < nvis && x.n0 + row < p.N)
-              gv[j] = __ldg(reinterpret_cast<const uint4*>(gbase + (size_t)row * p.dv));
-          }
-#pragma unroll
-          for (int j = 0; j < GB; ++j) {
-            const int row = et / cpr + (v0 + j) * rstep;
-            if (v0 + j >= nvis || x.n0 + row >= p.N) continue;
-            const uint32_t a = sbase + row * 128 + (((pc & 7) ^ (row & 7)) * 16);
-            const uint4 yv = ld_shared_v4(a);
-            const uint32_t yi[4] = {yv.x, yv.y, yv.z, yv.w};
-            const uint32_t gi[4] = {gv[j].x, gv[j].y, gv[j].z, gv[j].w};
-            uint32_t r[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              r[e] = pack_bf16(bf16lo_to_f32(yi[e]) * swishf(bf16lo_to_f32(gi[e])),
-                               bf16hi_to_f32(yi[e]) * swishf(bf16hi_to_f32(gi[e])));
-            st_shared_v4(a, r[0], r[1], r[2], r[3]);
-          }
-        }
-        xok = ok;
       }
       fence_proxy_async_smem();
       ok = epi_bar_and<EPI>(xok);
