@@ -145,7 +145,7 @@ def global_throughput(units_per_rank_per_step: float, steps: int, world: int, t_
 
 # Sources that decide what the chunk-output kernel does (its code, the
 # headers it includes and the tensor maps it is launched with).
-OUT_KERNEL_SOURCES = ("tc_out.cu", "sm100.cuh", "common.cuh", "kernels.h", "tmap.cu", "tmap.h")
+OUT_KERNEL_SOURCES = ("tc_out.cu", "sm100.cuh", "common.cuh", "tmap.cu", "tmap.h")
 
 
 def kernel_source_hash(names=OUT_KERNEL_SOURCES):
