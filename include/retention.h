@@ -263,6 +263,15 @@ RET_API int ret_last_cuda_error(void);
  */
 RET_API int ret_device_error(void);
 
+/*
+ * Self-test of the failure path above: launches one thread that waits on an
+ * mbarrier nothing will complete, with a limit of limit_ms (1 .. 10000).  The
+ * wait gives up, records site code 901 and the kernel returns, so the
+ * context stays usable; after the stream has run, ret_device_error() returns
+ * 901 (and clears it).  No GPU fault, trap or hang is involved.
+ */
+RET_API int ret_selftest_bounded_wait(int limit_ms, void* stream);
+
 /* Library version string (static storage). */
 RET_API const char* ret_version(void);
 

@@ -46,6 +46,7 @@ SIGNATURES = {
     "ret_last_cuda_error": (_I, []),
     "ret_version": (ctypes.c_char_p, []),
     "ret_device_error": (_I, []),
+    "ret_selftest_bounded_wait": (_I, [_I, _P]),
 }
 
 _lib = None

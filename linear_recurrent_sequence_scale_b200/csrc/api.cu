@@ -68,8 +68,15 @@ const char* ret_version(void) { return "retention-b200 0.1 (sm_100a)"; }
 int ret_device_error(void) {
   const int a = ret::tc_state_device_error();
   const int b = ret::tc_out_device_error();
-  if (a < 0 || b < 0) return -1;
-  return a ? a : b;
+  const int c = ret::selftest_device_error();
+  if (a < 0 || b < 0 || c < 0) return -1;
+  return a ? a : (b ? b : c);
+}
+
+int ret_selftest_bounded_wait(int limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 10000) return RET_EINVAL;
+  return cuda_status(
+      ret::launch_bounded_wait_selftest(limit_ms, static_cast<cudaStream_t>(stream)));
 }
 
 int ret_parallel_gated(const void* q, const void* k, const void* v, const float* gammas,

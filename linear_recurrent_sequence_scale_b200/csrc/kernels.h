@@ -56,5 +56,8 @@ cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const flo
                           cudaStream_t st);
 int tc_state_device_error();
 int tc_out_device_error();
+// Bounded-wait self-test (selftest.cu): a wait that runs out, site code 901.
+cudaError_t launch_bounded_wait_selftest(int limit_ms, cudaStream_t st);
+int selftest_device_error();
 
 }  // namespace ret

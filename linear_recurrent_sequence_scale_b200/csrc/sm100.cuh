@@ -90,17 +90,18 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site) {
+// Bounded wait for the phase with the given parity to complete: false (and
+// the site code recorded) after limit_ns, or at once if another wait failed.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    // give up at the time limit, or at once if another wait already failed
     if (*reinterpret_cast<volatile int*>(&g_device_error) != 0 ||
-        globaltimer() - t0 > kWaitLimitNs) {
+        globaltimer() - t0 > limit_ns) {
       record_error(site);
       return false;
     }

@@ -202,3 +202,8 @@ def test_backward_rejects_bad_arguments(lib):
     assert call(ws=None) == ret.RET_EWORKSPACE
     assert call(wsb=need - 1) == ret.RET_EWORKSPACE
     assert call(N=0, q=None, dO=None, gq=None, ds=None, ws=None, wsb=0) == ret.RET_OK
+
+
+def test_selftest_rejects_bad_limits(lib):
+    assert lib.ret_selftest_bounded_wait(0, None) == ret.RET_EINVAL
+    assert lib.ret_selftest_bounded_wait(20000, None) == ret.RET_EINVAL
