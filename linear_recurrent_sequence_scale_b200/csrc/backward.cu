@@ -119,6 +119,15 @@ __device__ __forceinline__ void stage_rows(float* dst, int ld, const T* src, int
   }
 }
 
+// Rows [r0, r0 + rows) of a float32 [.][d] state into smem (zeros past rows).
+__device__ __forceinline__ void stage_state_rows(float* dst, int ld, const float* src, int d,
+                                                 int r0, int rows) {
+  for (int e = threadIdx.x; e < TP * d; e += 256) {
+    const int r = e / d, x = e % d;
+    dst[r * ld + x] = r < rows ? src[(size_t)(r0 + r) * d + x] : 0.f;
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256)
 chunk_grad(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
@@ -134,6 +143,8 @@ chunk_grad(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
   float* b_k = b_v + TP * lv;      // [TP][dk+1]  other rows: K (A) / Q (B)
   float* ps = b_k + TP * lk;       // [TP][TP+1]
   float* ss = ps + TP * (TP + 1);  // [TP][TP+1]
+  const int li = (dk > dv ? dk : dv) + 1;
+  float* isum = ss + TP * (TP + 1);  // [TP][max(dk,dv)+1]: the cross-chunk terms
 
   const int bh = blockIdx.y;
   const float lg = log2f(gammas[bh % H]);
@@ -178,25 +189,30 @@ chunk_grad(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
       }
     }
   }
-  if (t < rows) {
-    const int n = p0 + t;
-    if (ci > 0 || has_r0) {  // + xi_n (R_{i-1} dO_n)
-      const float* R = rws + ((size_t)bh * nc + ci) * dk * dv;
-      const float xi = gpow(lg, n - cs + 1);
-#pragma unroll
-      for (int x = 0; x < MAXU; ++x) {
-        const int c = cg + 16 * x;
-        if (c < dk) {
-          float s = 0.f;
-          for (int j = 0; j < dv; ++j) s = fmaf(R[(size_t)c * dv + j], a_v[t * lv + j], s);
-          acc[x] = fmaf(xi, s, acc[x]);
-        }
+  // + xi_n (R_{i-1} dO_n): 16 rows of R at a time through shared memory
+  const bool has_r = ci > 0 || has_r0;
+  if (has_r) {
+    const float* R = rws + ((size_t)bh * nc + ci) * dk * dv;
+    const float xi = gpow(lg, p0 + t - cs + 1);
+    for (int cb = 0; cb < dk; cb += TP) {
+      __syncthreads();
+      stage_state_rows(b_v, lv, R, dv, cb, min(TP, dk - cb));
+      __syncthreads();
+      if (cb + cg < dk) {
+        float s = 0.f;
+        for (int j = 0; j < dv; ++j) s = fmaf(b_v[cg * lv + j], a_v[t * lv + j], s);
+        isum[t * li + cb + cg] = xi * s;
       }
     }
+    __syncthreads();
+  }
+  if (t < rows) {
+    const int n = p0 + t;
 #pragma unroll
     for (int x = 0; x < MAXU; ++x) {
       const int c = cg + 16 * x;
-      if (c < dk) Elem<T>::st(dq + ((size_t)bh * N + n) * dk + c, acc[x]);
+      if (c < dk)
+        Elem<T>::st(dq + ((size_t)bh * N + n) * dk + c, has_r ? acc[x] + isum[t * li + c] : acc[x]);
     }
   }
 
@@ -238,23 +254,50 @@ chunk_grad(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
       }
     }
   }
+  // + zeta_m (G v_m) and + zeta_m (G^T k_m), G = G_i staged 16 rows (then
+  // 16 columns) at a time
+  const float zeta = gpow(lg, L - 1 - (p0 + t - cs));
+  const float* G = gws + ((size_t)bh * nc + ci) * dk * dv;
+  for (int cb = 0; cb < dk; cb += TP) {
+    __syncthreads();
+    stage_state_rows(b_v, lv, G, dv, cb, min(TP, dk - cb));
+    __syncthreads();
+    if (cb + cg < dk) {
+      float s = 0.f;
+      for (int j = 0; j < dv; ++j) s = fmaf(b_v[cg * lv + j], a_v[t * lv + j], s);
+      isum[t * li + cb + cg] = zeta * s;
+    }
+  }
+  __syncthreads();
   if (t < rows) {
     const int m = p0 + t;
-    const float zeta = gpow(lg, L - 1 - (m - cs));
-    const float* G = gws + ((size_t)bh * nc + ci) * dk * dv;
 #pragma unroll
     for (int x = 0; x < MAXU; ++x) {
       const int c = cg + 16 * x;
-      if (c < dk) {  // + zeta_m (G v_m)
-        float s = 0.f;
-        for (int j = 0; j < dv; ++j) s = fmaf(G[(size_t)c * dv + j], a_v[t * lv + j], s);
-        Elem<T>::st(dk_ + ((size_t)bh * N + m) * dk + c, fmaf(zeta, s, acck[x]));
-      }
-      if (c < dv) {  // + zeta_m (G^T k_m)
-        float s = 0.f;
-        for (int i = 0; i < dk; ++i) s = fmaf(G[(size_t)i * dv + c], a_k[t * lk + i], s);
-        Elem<T>::st(dv_ + ((size_t)bh * N + m) * dv + c, fmaf(zeta, s, accv[x]));
-      }
+      if (c < dk) Elem<T>::st(dk_ + ((size_t)bh * N + m) * dk + c, acck[x] + isum[t * li + c]);
+    }
+  }
+  for (int cb = 0; cb < dv; cb += TP) {
+    __syncthreads();
+    // columns [cb, cb + 16) of G as rows of b_k: b_k[r][i] = G[i][cb + r]
+    for (int e = threadIdx.x; e < TP * dk; e += 256) {
+      const int r = e % TP, i = e / TP;
+      b_k[r * lk + i] = cb + r < dv ? G[(size_t)i * dv + cb + r] : 0.f;
+    }
+    __syncthreads();
+    if (cb + cg < dv) {
+      float s = 0.f;
+      for (int i = 0; i < dk; ++i) s = fmaf(b_k[cg * lk + i], a_k[t * lk + i], s);
+      isum[t * li + cb + cg] = zeta * s;
+    }
+  }
+  __syncthreads();
+  if (t < rows) {
+    const int m = p0 + t;
+#pragma unroll
+    for (int x = 0; x < MAXU; ++x) {
+      const int c = cg + 16 * x;
+      if (c < dv) Elem<T>::st(dv_ + ((size_t)bh * N + m) * dv + c, accv[x] + isum[t * li + c]);
     }
   }
 }
@@ -274,8 +317,8 @@ cudaError_t backward_t(const void* q, const void* k, const void* v, const float*
   grad_scan<T><<<g1, 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(dout), gammas,
                                    chunk, d_state_out, d_state_in, gws, H, N, dk, dv);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-  const size_t smem =
-      sizeof(float) * (size_t)(2 * TP * (dv + 1) + 2 * TP * (dk + 1) + 2 * TP * (TP + 1));
+  const size_t smem = sizeof(float) * (size_t)(2 * TP * (dv + 1) + 2 * TP * (dk + 1) +
+                                               2 * TP * (TP + 1) + TP * ((dk > dv ? dk : dv) + 1));
   auto fn = chunk_grad<T>;
   if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
       cudaSuccess)
