@@ -351,6 +351,60 @@ def test_chunkwise_backward_parity(torch_cuda, ret, case):
     assert _rel(gs, rs) <= (1e-5 if dt == "f32" else 1e-4)
 
 
+# --- the largest supported sizes and many (batch, head) pairs -------------------
+
+EDGE_CASES = [
+    # form, dtype, B, H, N, dk, dv, chunk, gn_eps
+    ("chunkwise", "bf16", 1, 1, 300, 512, 512, 100, 1e-5),   # d = 512: CUDA-core path
+    ("chunkwise", "f32", 1, 1, 150, 512, 64, 64, None),
+    ("parallel", "f32", 1, 1, 96, 512, 512, None, 1e-5),
+    ("chunkwise", "bf16", 64, 32, 17, 64, 64, 128, 1e-5),    # 2048 pairs, one short chunk
+    ("parallel", "bf16", 64, 32, 9, 128, 128, None, None),
+]
+
+
+@pytest.mark.parametrize("case", EDGE_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_edge_sizes(torch_cuda, ret, case):
+    torch = torch_cuda
+    form, dt, B, H, N, dk, dv, chunk, gn = case
+    gam = [1.0 - 2.0 ** (-5 - (h % 12)) for h in range(H)]
+    inp = wl.make_inputs(B, H, N, dk, dv, dt, seed=111 + N + dk, with_state=(form == "chunkwise"),
+                         gammas=gam)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    if form == "chunkwise":
+        o, s = ret.chunkwise(q, k, v, g, chunk, state_in=_dev(inp["state"]), return_state=True,
+                             gn_eps=gn)
+        torch.cuda.synchronize()
+        o_ref, s_ref = _ref_chunkwise(inp, chunk, gn, True)
+        assert _rel(s, s_ref) <= STATE_TOL
+    else:
+        o = ret.parallel(q, k, v, g, gn_eps=gn)
+        torch.cuda.synchronize()
+        o_ref, _ = oracle.parallel(inp["q"].exact, inp["k"].exact, inp["v"].exact, inp["gammas"])
+        if gn is not None:
+            o_ref = oracle.group_norm(o_ref, gn)
+    assert _rel(o, o_ref) <= TOL[dt]
+
+
+@pytest.mark.parametrize("dk,dv", [(4096, 64), (256, 1024)])
+def test_step_largest_sizes(torch_cuda, ret, dk, dv):
+    """The decode step at its limits: d_k 4096, and d_v 1024 with GroupNorm
+    over a cluster of 8 CTAs."""
+    torch = torch_cuda
+    B, H = 2, 2
+    inp = wl.make_inputs(B, H, 1, dk, dv, "bf16", seed=121 + dk, with_state=True)
+    state = _dev(inp["state"])
+    o = ret.step(_dev(inp["q"])[:, :, 0].contiguous(), _dev(inp["k"])[:, :, 0].contiguous(),
+                 _dev(inp["v"])[:, :, 0].contiguous(), _gam(torch, inp["gammas"]), state,
+                 gn_eps=1e-5)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.step(inp["q"].exact[:, :, 0], inp["k"].exact[:, :, 0],
+                               inp["v"].exact[:, :, 0], inp["gammas"], inp["state"].exact)
+    assert _rel(o, oracle.group_norm(o_ref, 1e-5)) <= TOL["bf16"]
+    assert _rel(state, s_ref) <= STATE_TOL
+
+
 # --- parallel form -----------------------------------------------------------------
 
 PAR_CASES = [
