@@ -12,6 +12,9 @@
 // stores them.  The partial q.S sums of the 8 warps meet in shared memory.
 // With GroupNorm the CTAs of one (b, h) form a thread-block cluster and
 // exchange their row statistics through distributed shared memory.
+// Consecutive steps on a stream use programmatic dependent launch: a step's
+// CTAs are scheduled while the previous step drains and wait (griddepcontrol)
+// until its writes are visible, which hides the launch gap between steps.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -51,6 +54,10 @@ step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   __shared__ float scratch[8];
   __shared__ float stats[2];              // this CTA's partial sum, sum of squares
 
+  // the previous grid on the stream (e.g. the step before) must be complete
+  // before anything is read; the next one may be scheduled from now on
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int bh = blockIdx.y;
   const int h = bh % H;
   const int c0 = blockIdx.x * STEP_COLS;
@@ -151,32 +158,34 @@ static cudaError_t launch_step_t(const void* q, const void* k, const void* v, co
   const T* vv = static_cast<const T*>(v);
   T* oo = static_cast<T*>(o);
   const T* gg = static_cast<const T*>(gate);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(STEP_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = nct;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
   if (eps < 0.f) {
     auto fn = step_kernel<T, false>;
     if (smem > 48 * 1024) {
       cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
-    fn<<<grid, STEP_THREADS, smem, st>>>(qq, kk, vv, gammas, state, gg, oo, H, dk, dv, eps);
-    return cudaPeekAtLastError();
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fn, qq, kk, vv, gammas, state, gg, oo, H, dk, dv, eps);
   }
   auto fn = step_kernel<T, true>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = dim3(STEP_THREADS);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = nct;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, fn, qq, kk, vv, gammas, state, gg, oo, H, dk, dv, eps);
 }
 
