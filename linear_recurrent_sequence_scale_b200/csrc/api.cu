@@ -93,7 +93,7 @@ int ret_parallel_gated(const void* q, const void* k, const void* v, const float*
   if (dtype == RET_BF16 && tc_dims(dk, dv)) {
     if ((int64_t)((N + 127) / 128) > 65535) return RET_EUNSUPPORTED;
     return cuda_status(ret::launch_tc_out(q, k, v, gammas, 0, nullptr, 0, gate, o, B, H, N, dk,
-                                          dv, gn_eps, 1, st));
+                                          dv, gn_eps, 1, 0, st));
   }
   return cuda_status(ret::launch_simt_parallel(q, k, v, gammas, gate, o, B, H, N, dk, dv, dtype,
                                                gn_eps, st));
@@ -173,10 +173,16 @@ int ret_chunkwise_states(const void* k, const void* v, const float* gammas, int 
                                              dk, dv, dtype, workspace, st));
 }
 
-int ret_chunkwise_output_gated(const void* q, const void* k, const void* v, const float* gammas,
-                               int chunk, int has_state_in, const void* gate, void* o, int B,
-                               int H, int N, int dk, int dv, int dtype, float gn_eps,
-                               const void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// The output phase; after_states: the states phase of the same call was
+// launched just before it on the stream (programmatic dependent launch).
+int chunkwise_output_impl(const void* q, const void* k, const void* v, const float* gammas,
+                          int chunk, int has_state_in, const void* gate, void* o, int B, int H,
+                          int N, int dk, int dv, int dtype, float gn_eps, const void* workspace,
+                          size_t workspace_bytes, void* stream, bool after_states) {
   int s = check_chunkwise(B, H, N, dk, dv, dtype, chunk, gammas, workspace, workspace_bytes);
   if (s) return s;
   if ((s = check_eps(gn_eps))) return s;
@@ -187,9 +193,21 @@ int ret_chunkwise_output_gated(const void* q, const void* k, const void* v, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tc_config(dtype, dk, dv, chunk))
     return cuda_status(ret::launch_tc_out(q, k, v, gammas, chunk, workspace, has_state_in != 0,
-                                          gate, o, B, H, N, dk, dv, gn_eps, 0, st));
+                                          gate, o, B, H, N, dk, dv, gn_eps, 0, after_states, st));
   return cuda_status(ret::launch_simt_output(q, k, v, gammas, chunk, gate, o, B, H, N, dk, dv,
                                              dtype, gn_eps, workspace, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int ret_chunkwise_output_gated(const void* q, const void* k, const void* v, const float* gammas,
+                               int chunk, int has_state_in, const void* gate, void* o, int B,
+                               int H, int N, int dk, int dv, int dtype, float gn_eps,
+                               const void* workspace, size_t workspace_bytes, void* stream) {
+  return chunkwise_output_impl(q, k, v, gammas, chunk, has_state_in, gate, o, B, H, N, dk, dv,
+                               dtype, gn_eps, workspace, workspace_bytes, stream, false);
 }
 
 int ret_chunkwise_output(const void* q, const void* k, const void* v, const float* gammas,
@@ -218,8 +236,11 @@ int ret_chunkwise_gated(const void* q, const void* k, const void* v, const float
   s = ret_chunkwise_states(k, v, gammas, chunk, state_in, state_out, B, H, N, dk, dv, dtype,
                            workspace, workspace_bytes, stream);
   if (s) return s;
-  return ret_chunkwise_output_gated(q, k, v, gammas, chunk, state_in != nullptr, gate, o, B, H, N,
-                                    dk, dv, dtype, gn_eps, workspace, workspace_bytes, stream);
+  // the states kernel ran (and may still be draining) unless nothing needed it
+  const bool scanned = tc_config(dtype, dk, dv, chunk) &&
+                       ((N + chunk - 1) / chunk > 1 || state_out || state_in);
+  return chunkwise_output_impl(q, k, v, gammas, chunk, state_in != nullptr, gate, o, B, H, N, dk,
+                               dv, dtype, gn_eps, workspace, workspace_bytes, stream, scanned);
 }
 
 int ret_chunkwise(const void* q, const void* k, const void* v, const float* gammas, int chunk,

@@ -53,7 +53,7 @@ cudaError_t launch_tc_state(const void* k, const void* v, const float* gammas, i
 cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const float* gammas,
                           int chunk, const void* ws, int has_state0, const void* gate, void* o,
                           int B, int H, int N, int dk, int dv, float eps, int parallel_form,
-                          cudaStream_t st);
+                          int after_states, cudaStream_t st);
 int tc_state_device_error();
 int tc_out_device_error();
 // Bounded-wait self-test (selftest.cu): a wait that runs out, site code 901.

@@ -286,6 +286,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
       // stages to issue: it polls between stages and waits only when the tile
       // that needs the Q starts.
       int qn = 0;  // next Q to load (tile sequence number)
+      bool r_ready = false;
       auto issue_q = [&](bool block) -> bool {
         const int tile = tile_at(p, qn);
         if (tile < 0 || qn > k + (NQB - 1)) return true;
@@ -339,6 +340,13 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           }
         }
         if (x.has_r && ok) {
+          if (!r_ready) {
+            // The chunk states come from the state scan launched just before
+            // this kernel (programmatic dependent launch): this grid may have
+            // started while it drained; wait for it before the first read.
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            r_ready = true;
+          }
           const int zr = x.bh * p.nc + x.ci;
           for (int s = 0; s < kq && ok; ++s, ++g) {
             uint64_t* bar;
@@ -712,7 +720,7 @@ int tc_out_device_error() { return read_clear_device_error(); }
 cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const float* gammas,
                           int chunk, const void* ws, int has_state0, const void* gate, void* o,
                           int B, int H, int N, int dk, int dv, float eps, int parallel_form,
-                          cudaStream_t st) {
+                          int after_states, cudaStream_t st) {
   using namespace k3;
   const uint64_t BH = (uint64_t)B * H;
   Params p;
@@ -768,13 +776,18 @@ cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const flo
   cfg.blockDim = dim3(eps >= 0.f ? threads<true>() : threads<false>());
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = p.nslices;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  // After the state scan of the same call, the grid may be scheduled while
+  // that scan drains (it only waits before reading the chunk states); any
+  // other launch keeps full stream order.
+  cfg.numAttrs = after_states ? 2 : 1;
   // Short tiles (chunkwise) gain most from loading the next Q early; long
   // tiles (parallel form) from a deeper ring (both measured on B200).
   const int nqb = parallel_form ? 1 : 2;

@@ -97,6 +97,9 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
   const uint32_t rcol = static_cast<uint32_t>(p.mh * p.nt);
   const uint32_t tmem_cols = 2 * rcol;     // 128, 256 or 512
 
+  // the chunk-output kernel of the same call may be scheduled once every CTA
+  // of this grid runs (it waits for this grid before reading the states)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
