@@ -9,8 +9,9 @@
 // Persistent kernel.  A work tile is a 128-row query tile of one chunk and a
 // slice of up to 256 output columns; d_v = 512 runs two slices as a 2-CTA
 // cluster that exchanges GroupNorm row statistics through distributed shared
-// memory.  Each CTA (one per SM) walks tiles in a fixed round-robin order and
-// overlaps consecutive tiles:
+// memory.  Each CTA (one per SM) walks its tiles in a fixed order (the row
+// tiles of a chunk back to back when there are enough chunks, see tile_at)
+// and overlaps consecutive tiles:
 //   warp 0     TMA: Q of the next tile into the second of two Q buffers while
 //              the current tile runs; K, V and R_{i-1} tiles through a 3-stage
 //              ring of 32 KB stages, in the order the MMAs consume them
@@ -20,12 +21,16 @@
 //              back into the first 64 columns of S_t's TMEM buffer; then
 //              Q (.) xi in place in the tile's Q buffer
 //   warps 6-   epilogue (4 warps, or with GroupNorm 8: two per TMEM lane
-//              quadrant, each on half of the columns): read O from TMEM,
-//              optional GroupNorm (Chan's merge of per-32-column statistics,
-//              of the two halves through shared memory, then one exchange
-//              with the peer CTA), bf16 rows staged in the tile's Q buffer and
-//              written by TMA; O is freed for the next tile's P V after the
-//              last TMEM read
+//              quadrant, each on half of the columns): one pass over O in
+//              TMEM, after which O is free for the next tile's P V; with
+//              GroupNorm the per-32-column statistics (Chan's merge, the two
+//              halves through shared memory, one exchange with the peer CTA)
+//              and the deviations held as scaled f16 in registers; bf16 rows
+//              staged in the tile's Q buffer (with the optional output gate
+//              loaded there by TMA and applied in place) and written by TMA
+// When it follows the state scan of the same call the kernel is launched as
+// a programmatic dependent: it may start while the scan drains, and the
+// loader waits for the scan (griddepcontrol.wait) before the first R_{i-1}.
 // The decay mask is never stored: each thread walks its row from the highest
 // column down, multiplying by gamma per column, one exp2 per 32 columns.
 // S_t's buffer is rewritten by Q K_{t+2}^T only after the MMA reading P_t was

@@ -203,6 +203,7 @@ GATED_CASES = [
     # form, dtype, B, H, N, dk, dv, chunk, gn_eps
     ("chunkwise", "bf16", 1, 2, 1000, 256, 512, 512, 1e-5),   # tensor cores, 2 d_v slices
     ("chunkwise", "bf16", 2, 2, 333, 128, 128, 128, None),    # tensor cores, ragged tail
+    ("chunkwise", "bf16", 1, 2, 300, 64, 64, 128, 1e-5),      # one 64-column box per slice
     ("parallel", "bf16", 1, 3, 300, 64, 256, None, 1e-5),
     ("chunkwise", "f32", 1, 2, 200, 64, 96, 64, 1e-5),        # SIMT path
     ("parallel", "f32", 1, 2, 130, 32, 40, None, None),
@@ -250,6 +251,23 @@ def test_gated_step_parity(torch_cuda, ret, gn):
         y_ref = oracle.group_norm(y_ref, gn)
     assert _rel(o, oracle.gated(y_ref, gate.exact)) <= TOL["bf16"]
     assert _rel(state, s_ref) <= STATE_TOL
+
+
+def test_gated_output_phase(torch_cuda, ret):
+    """The gate through the two-phase form (ret_chunkwise_output_gated)."""
+    torch = torch_cuda
+    B, H, N, dk, dv, C = 1, 2, 600, 128, 256, 256
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=73, with_state=True)
+    gate = wl.from_values(np.random.default_rng(74).standard_normal((B, H, N, dv)), "bf16")
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    ws = torch.empty(ret.chunkwise_workspace_bytes(B, H, N, dk, dv, C, q.dtype),
+                     dtype=torch.uint8, device="cuda")
+    ret.chunkwise_states(k, v, g, C, ws, state_in=_dev(inp["state"]))
+    o = ret.chunkwise_output(q, k, v, g, C, ws, has_state_in=True, gn_eps=1e-5, gate=_dev(gate))
+    torch.cuda.synchronize()
+    y_ref, _ = _ref_chunkwise(inp, C, 1e-5, True)
+    assert _rel(o, oracle.gated(y_ref, gate.exact)) <= TOL["bf16"]
 
 
 def test_gate_none_is_the_ungated_call(torch_cuda, ret):
