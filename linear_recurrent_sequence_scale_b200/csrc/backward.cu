@@ -14,7 +14,9 @@
 // and the gradient of the incoming state is G_{-1}.
 //   1. the forward chunk states R_{i-1} (the chunkwise states phase, float32)
 //   2. grad_scan: G_i for every chunk, walking the chunks backwards
-//   3. chunk_grad: per (b, h, chunk, 16 positions) the three row gradients.
+//   3. chunk_grad: per (b, h, chunk, 16 positions) the in-chunk parts of the
+//      three row gradients
+//   4. cross_chunk_gemm: the cross-chunk parts, one batched GEMM each.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -119,20 +121,10 @@ __device__ __forceinline__ void stage_rows(float* dst, int ld, const T* src, int
   }
 }
 
-// Rows [r0, r0 + rows) of a float32 [.][d] state into smem (zeros past rows).
-__device__ __forceinline__ void stage_state_rows(float* dst, int ld, const float* src, int d,
-                                                 int r0, int rows) {
-  for (int e = threadIdx.x; e < TP * d; e += 256) {
-    const int r = e / d, x = e % d;
-    dst[r * ld + x] = r < rows ? src[(size_t)(r0 + r) * d + x] : 0.f;
-  }
-}
-
 template <typename T>
 __global__ void __launch_bounds__(256)
 chunk_grad(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
            const T* __restrict__ dout, const float* __restrict__ gammas, int chunk,
-           const float* __restrict__ rws, int has_r0, const float* __restrict__ gws,
            T* __restrict__ dq, T* __restrict__ dk_, T* __restrict__ dv_, int H, int N, int dk,
            int dv) {
   extern __shared__ float sm[];
@@ -143,8 +135,6 @@ chunk_grad(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
   float* b_k = b_v + TP * lv;      // [TP][dk+1]  other rows: K (A) / Q (B)
   float* ps = b_k + TP * lk;       // [TP][TP+1]
   float* ss = ps + TP * (TP + 1);  // [TP][TP+1]
-  const int li = (dk > dv ? dk : dv) + 1;
-  float* isum = ss + TP * (TP + 1);  // [TP][max(dk,dv)+1]: the cross-chunk terms
 
   const int bh = blockIdx.y;
   const float lg = log2f(gammas[bh % H]);
@@ -155,8 +145,6 @@ chunk_grad(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
   const int ce = min(N, cs + chunk);
   if (p0 >= ce) return;
   const int rows = min(TP, ce - p0);
-  const int L = ce - cs;
-  const int nc = cdiv(N, chunk);
   const int tid = threadIdx.x;
   const int t = tid & 15, cg = tid >> 4;  // accumulation: row t, columns cg + 16 x
   const int da = tid >> 4, db = tid & 15;  // dot products: pair (da, db)
@@ -189,30 +177,12 @@ chunk_grad(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
       }
     }
   }
-  // + xi_n (R_{i-1} dO_n): 16 rows of R at a time through shared memory
-  const bool has_r = ci > 0 || has_r0;
-  if (has_r) {
-    const float* R = rws + ((size_t)bh * nc + ci) * dk * dv;
-    const float xi = gpow(lg, p0 + t - cs + 1);
-    for (int cb = 0; cb < dk; cb += TP) {
-      __syncthreads();
-      stage_state_rows(b_v, lv, R, dv, cb, min(TP, dk - cb));
-      __syncthreads();
-      if (cb + cg < dk) {
-        float s = 0.f;
-        for (int j = 0; j < dv; ++j) s = fmaf(b_v[cg * lv + j], a_v[t * lv + j], s);
-        isum[t * li + cb + cg] = xi * s;
-      }
-    }
-    __syncthreads();
-  }
   if (t < rows) {
     const int n = p0 + t;
 #pragma unroll
     for (int x = 0; x < MAXU; ++x) {
       const int c = cg + 16 * x;
-      if (c < dk)
-        Elem<T>::st(dq + ((size_t)bh * N + n) * dk + c, has_r ? acc[x] + isum[t * li + c] : acc[x]);
+      if (c < dk) Elem<T>::st(dq + ((size_t)bh * N + n) * dk + c, acc[x]);
     }
   }
 
@@ -254,50 +224,88 @@ chunk_grad(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
       }
     }
   }
-  // + zeta_m (G v_m) and + zeta_m (G^T k_m), G = G_i staged 16 rows (then
-  // 16 columns) at a time
-  const float zeta = gpow(lg, L - 1 - (p0 + t - cs));
-  const float* G = gws + ((size_t)bh * nc + ci) * dk * dv;
-  for (int cb = 0; cb < dk; cb += TP) {
-    __syncthreads();
-    stage_state_rows(b_v, lv, G, dv, cb, min(TP, dk - cb));
-    __syncthreads();
-    if (cb + cg < dk) {
-      float s = 0.f;
-      for (int j = 0; j < dv; ++j) s = fmaf(b_v[cg * lv + j], a_v[t * lv + j], s);
-      isum[t * li + cb + cg] = zeta * s;
-    }
-  }
-  __syncthreads();
   if (t < rows) {
     const int m = p0 + t;
 #pragma unroll
     for (int x = 0; x < MAXU; ++x) {
       const int c = cg + 16 * x;
-      if (c < dk) Elem<T>::st(dk_ + ((size_t)bh * N + m) * dk + c, acck[x] + isum[t * li + c]);
+      if (c < dk) Elem<T>::st(dk_ + ((size_t)bh * N + m) * dk + c, acck[x]);
+      if (c < dv) Elem<T>::st(dv_ + ((size_t)bh * N + m) * dv + c, accv[x]);
     }
   }
-  for (int cb = 0; cb < dv; cb += TP) {
+}
+
+// Cross-chunk terms as one batched GEMM per (b, h, chunk), added to the
+// rows chunk_grad wrote:
+//     out[n] += s_n * (A[n] . S')    over the chunk's positions n,
+// with S' = S^T (TRANS: dQ += xi (.) dO R_{i-1}^T, dK += zeta (.) V G_i^T) or
+// S' = S (dV += zeta (.) K G_i), S a float32 [dk][dv] chunk state.  Tiles of
+// 64 rows x 64 columns, 4 x 4 results per thread, 16-deep slices of A and S'
+// through shared memory.
+constexpr int GM = 64, GN_ = 64, GK = 16;
+
+template <typename T, bool TRANS, bool XI>
+__global__ void __launch_bounds__(256)
+cross_chunk_gemm(const T* __restrict__ a, const float* __restrict__ states, int has_r0,
+                 const float* __restrict__ gammas, int chunk, T* __restrict__ out, int H, int N,
+                 int ka, int ncol, int dk, int dv) {
+  __shared__ float as[GK][GM + 4];
+  __shared__ float bs[GK][GN_ + 4];
+  const int nc = cdiv(N, chunk);
+  const int rpc = cdiv(chunk, GM);        // row blocks per chunk
+  const int ci = blockIdx.y / rpc;
+  const int cs = ci * chunk;
+  const int r0 = cs + (blockIdx.y % rpc) * GM;
+  const int ce = min(N, cs + chunk);
+  if (r0 >= ce || (XI && ci == 0 && !has_r0)) return;
+  const int bh = blockIdx.z;
+  const int c0 = blockIdx.x * GN_;
+  const float lg = log2f(gammas[bh % H]);
+  const float* S = states + ((size_t)bh * nc + ci) * dk * dv;
+  const int tid = threadIdx.x;
+  const int ty = tid >> 4, tx = tid & 15;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < ka; k0 += GK) {
     __syncthreads();
-    // columns [cb, cb + 16) of G as rows of b_k: b_k[r][i] = G[i][cb + r]
-    for (int e = threadIdx.x; e < TP * dk; e += 256) {
-      const int r = e % TP, i = e / TP;
-      b_k[r * lk + i] = cb + r < dv ? G[(size_t)i * dv + cb + r] : 0.f;
+    for (int e = tid; e < GM * GK; e += 256) {  // A rows r0.., columns k0..
+      const int r = e / GK, kk = e % GK;
+      const int n = r0 + r;
+      as[kk][r] = (n < ce && k0 + kk < ka) ? Elem<T>::ld(a + ((size_t)bh * N + n) * ka + k0 + kk)
+                                           : 0.f;
+    }
+    for (int e = tid; e < GK * GN_; e += 256) {  // S' rows k0.., columns c0..
+      int kk, c;
+      if (TRANS) { c = e / GK; kk = e % GK; } else { kk = e / GN_; c = e % GN_; }
+      float x = 0.f;
+      if (k0 + kk < ka && c0 + c < ncol)
+        x = TRANS ? S[(size_t)(c0 + c) * dv + k0 + kk] : S[(size_t)(k0 + kk) * dv + c0 + c];
+      bs[kk][c] = x;
     }
     __syncthreads();
-    if (cb + cg < dv) {
-      float s = 0.f;
-      for (int i = 0; i < dk; ++i) s = fmaf(b_k[cg * lk + i], a_k[t * lk + i], s);
-      isum[t * li + cb + cg] = zeta * s;
-    }
-  }
-  __syncthreads();
-  if (t < rows) {
-    const int m = p0 + t;
 #pragma unroll
-    for (int x = 0; x < MAXU; ++x) {
-      const int c = cg + 16 * x;
-      if (c < dv) Elem<T>::st(dv_ + ((size_t)bh * N + m) * dv + c, accv[x] + isum[t * li + c]);
+    for (int kk = 0; kk < GK; ++kk) {
+      float av[4], bv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) av[i] = as[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = bs[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+  }
+  const int L = ce - cs;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int n = r0 + ty * 4 + i;
+    if (n >= ce) continue;
+    const float sc = XI ? gpow(lg, n - cs + 1) : gpow(lg, L - 1 - (n - cs));
+    T* orow = out + ((size_t)bh * N + n) * ncol;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = c0 + tx * 4 + j;
+      if (c < ncol) Elem<T>::st(orow + c, Elem<T>::ld(orow + c) + sc * acc[i][j]);
     }
   }
 }
@@ -317,8 +325,8 @@ cudaError_t backward_t(const void* q, const void* k, const void* v, const float*
   grad_scan<T><<<g1, 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(dout), gammas,
                                    chunk, d_state_out, d_state_in, gws, H, N, dk, dv);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-  const size_t smem = sizeof(float) * (size_t)(2 * TP * (dv + 1) + 2 * TP * (dk + 1) +
-                                               2 * TP * (TP + 1) + TP * ((dk > dv ? dk : dv) + 1));
+  const size_t smem =
+      sizeof(float) * (size_t)(2 * TP * (dv + 1) + 2 * TP * (dk + 1) + 2 * TP * (TP + 1));
   auto fn = chunk_grad<T>;
   if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
       cudaSuccess)
@@ -326,8 +334,18 @@ cudaError_t backward_t(const void* q, const void* k, const void* v, const float*
   dim3 g2(nc * cdiv(chunk, TP), B * H);
   fn<<<g2, 256, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
                             static_cast<const T*>(v), static_cast<const T*>(dout), gammas, chunk,
-                            rws, state_in != nullptr, gws, static_cast<T*>(dq),
+                            static_cast<T*>(dq),
                             static_cast<T*>(dk_), static_cast<T*>(dv_), H, N, dk, dv);
+  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  const int rb = nc * cdiv(chunk, GM);
+  const dim3 gq(cdiv(dk, GN_), rb, B * H), gv_(cdiv(dv, GN_), rb, B * H);
+  cross_chunk_gemm<T, true, true><<<gq, 256, 0, st>>>(
+      static_cast<const T*>(dout), rws, state_in != nullptr, gammas, chunk, static_cast<T*>(dq), H,
+      N, dv, dk, dk, dv);
+  cross_chunk_gemm<T, true, false><<<gq, 256, 0, st>>>(
+      static_cast<const T*>(v), gws, 1, gammas, chunk, static_cast<T*>(dk_), H, N, dv, dk, dk, dv);
+  cross_chunk_gemm<T, false, false><<<gv_, 256, 0, st>>>(
+      static_cast<const T*>(k), gws, 1, gammas, chunk, static_cast<T*>(dv_), H, N, dk, dv, dk, dv);
   return cudaPeekAtLastError();
 }
 
