@@ -14,7 +14,8 @@ Pages cited (by title; the web pages on retention this build follows):
   [glossary]     "RetNet" entry of the jisaku.com glossary (efficient-arch-
                  retnet): definition of D, the three modes, FAQ Q2.
   [Spiral.AI]    "RetNet入門" (Spiral.AI Tech Blog, news.ainew.jp digest),
-                 section Multi-Scale Retention (MSR).
+                 sections Multi-Scale Retention (MSR) and the one on other
+                 non-Transformer architectures (LEX Transformer, xPos).
   [Medium]       "What Is RetNet ? could it challenge the dominance of the
                  Transformer ?" (Medium, Publicis Sapient), section "How is
                  this dual representation achieved?".
@@ -42,6 +43,12 @@ in the design notes):
     product (the Medium page mentions three such factors without formulas).
   * Gate: the block's "swish gating" is read as swish(G) (.) Y with the gate
     G supplied by the caller, swish(x) = x sigmoid(x).
+  * xPos rotation: the pages call it a complex rotation of Q and K that
+    carries relative position, and give no formula.  Read as: channels
+    (2c, 2c+1) of a row are the real and imaginary parts of z_c, and the row
+    at position n is multiplied by e^{i n theta_c}; the angles theta are
+    supplied by the caller (the pages give no values); no length scaling
+    (the decay gamma already plays that role in retention).
 """
 from __future__ import annotations
 
@@ -217,6 +224,32 @@ def gated(y, g):
     of the operator; the projection that produces it and the output
     projection after the gate belong to the layer around it."""
     return swish(g) * _f64(y)
+
+
+def rotate(x, theta, pos0: int = 0):
+    """xPos-style rotation of q or k ([RetNet blog] core components, item 3:
+    a complex rotation that puts relative position into Q and K; [Spiral.AI]
+    LEX Transformer paragraph: the xPos term that links the recurrent and the
+    parallel forms).
+
+    x [..., N, d] with d even, theta [d/2]; the row at index j has position
+    n = pos0 + j.  With phi = n theta_c, channel pair c turns by phi:
+        y[2c]   = x[2c] cos(phi) - x[2c+1] sin(phi)
+        y[2c+1] = x[2c] sin(phi) + x[2c+1] cos(phi)
+    Rotating both q and k this way makes q'_n . k'_m = Re sum_c
+    z_c(q_n) conj(z_c(k_m)) e^{i (n-m) theta_c}, a function of n - m only."""
+    x = _f64(x)
+    d = x.shape[-1]
+    if d % 2:
+        raise ValueError("rotate needs an even row length")
+    n = pos0 + np.arange(x.shape[-2], dtype=np.float64)
+    phi = n[:, None] * _f64(theta)[None, :]          # [N, d/2]
+    c, s = np.cos(phi), np.sin(phi)
+    re, im = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = re * c - im * s
+    y[..., 1::2] = re * s + im * c
+    return y
 
 
 def rel_frobenius(x, ref) -> float:

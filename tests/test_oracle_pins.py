@@ -406,3 +406,96 @@ def test_page_chunk_state_exact_only_for_gamma_one():
     o_m, s_m = _chunkwise_mutant(q, k, v, [1.0], 4, "page_chunk_state")
     assert oracle.rel_frobenius(o_m, o_ref) < 1e-12
     assert oracle.rel_frobenius(s_m, s_ref) < 1e-12
+
+
+# --- xPos rotation ---------------------------------------------------------------
+
+def test_hand_worked_rotation():
+    g = _golden()["rotation"]
+    theta = np.pi * np.asarray(g["theta_over_pi"])
+    y = oracle.rotate(np.asarray(g["x"], dtype=np.float64), theta, g["pos0"])
+    np.testing.assert_allclose(y, g["y"], rtol=0, atol=1e-14)
+
+
+def _rotation_pins_hold(rot):
+    """The rotation pins, for the oracle or a planted mutant: the hand-worked
+    rows, complex multiplication by e^{i n theta} done with numpy's complex
+    type, and q'_n . k'_m depending on n - m only."""
+    g = _golden()["rotation"]
+    theta = np.pi * np.asarray(g["theta_over_pi"])
+    ok = np.allclose(rot(np.asarray(g["x"], dtype=np.float64), theta, g["pos0"]), g["y"],
+                     rtol=0, atol=1e-12)
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((2, 3, 7, 10))
+    th = rng.uniform(0.0, 2.0, 5)
+    z = (x[..., 0::2] + 1j * x[..., 1::2]) * np.exp(1j * np.outer(np.arange(5, 12), th))
+    want = np.stack([z.real, z.imag], axis=-1).reshape(x.shape)
+    ok = ok and np.allclose(rot(x, th, 5), want, rtol=0, atol=1e-12)
+    q, k = rng.standard_normal((1, 6)), rng.standard_normal((1, 6))
+    th = rng.uniform(0.0, 2.0, 3)
+    dots = [float(rot(q, th, n)[0] @ rot(k, th, m)[0]) for n, m in [(4, 1), (9, 6), (3, 0)]]
+    ok = ok and np.allclose(dots, dots[0], rtol=1e-12)
+    return ok
+
+
+def test_rotation_pins():
+    assert _rotation_pins_hold(oracle.rotate)
+
+
+def test_rotation_invariants():
+    """theta = 0 and position 0 leave rows unchanged; each channel pair keeps
+    its length; turning by theta1 then theta2 is turning by theta1 + theta2;
+    rotating q and k with the same offset leaves retention unchanged, since
+    q'_n . k'_m depends on n - m only."""
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((2, 2, 9, 8))
+    t1, t2 = rng.uniform(-3, 3, 4), rng.uniform(-3, 3, 4)
+    np.testing.assert_array_equal(oracle.rotate(x, np.zeros(4), 17), x)
+    np.testing.assert_allclose(oracle.rotate(x[..., :1, :], t1, 0), x[..., :1, :], rtol=0,
+                               atol=0)
+    y = oracle.rotate(x, t1, 3)
+    np.testing.assert_allclose(y[..., 0::2] ** 2 + y[..., 1::2] ** 2,
+                               x[..., 0::2] ** 2 + x[..., 1::2] ** 2, rtol=1e-13)
+    np.testing.assert_allclose(oracle.rotate(oracle.rotate(x, t1, 3), t2, 3),
+                               oracle.rotate(x, t1 + t2, 3), rtol=0, atol=1e-12)
+    q, k, v, _ = _rand(rng, 1, 2, 12, 8, 3, state=False)
+    gam = [0.9, 0.6]
+    o0, _ = oracle.parallel(oracle.rotate(q, t1, 0), oracle.rotate(k, t1, 0), v, gam)
+    o1, _ = oracle.parallel(oracle.rotate(q, t1, 1000), oracle.rotate(k, t1, 1000), v, gam)
+    assert oracle.rel_frobenius(o1, o0) < 1e-12
+    with pytest.raises(ValueError):
+        oracle.rotate(np.zeros((2, 3)), np.zeros(1))
+
+
+def _rotate_mutant(x, theta, pos0, mutation):
+    """A copy of the oracle's rotation with one planted mistake."""
+    x = np.asarray(x, dtype=np.float64)
+    half = x.shape[-1] // 2
+    n = pos0 + np.arange(x.shape[-2], dtype=np.float64)
+    if mutation == "position_off_by_one":
+        n = n + 1
+    phi = n[:, None] * np.asarray(theta, dtype=np.float64)[None, :]
+    if mutation == "negative_angle":
+        phi = -phi
+    c, s = np.cos(phi), np.sin(phi)
+    if mutation == "cos_sin_swapped":
+        c, s = s, c
+    if mutation == "half_split_pairs":
+        re, im = x[..., :half], x[..., half:]
+    else:
+        re, im = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    if mutation == "half_split_pairs":
+        y[..., :half], y[..., half:] = re * c - im * s, re * s + im * c
+    else:
+        y[..., 0::2], y[..., 1::2] = re * c - im * s, re * s + im * c
+    if mutation == "rows_not_positions":       # every row turned by pos0 alone
+        y[..., 0::2] = re * np.cos(pos0 * theta) - im * np.sin(pos0 * theta)
+        y[..., 1::2] = re * np.sin(pos0 * theta) + im * np.cos(pos0 * theta)
+    return y
+
+
+@pytest.mark.parametrize("mutation", ["position_off_by_one", "negative_angle", "cos_sin_swapped",
+                                      "half_split_pairs", "rows_not_positions"])
+def test_rotation_pins_catch_planted_mistakes(mutation):
+    assert not _rotation_pins_hold(lambda x, t, p: _rotate_mutant(x, t, p, mutation))
