@@ -24,6 +24,8 @@ is needed between steps.  The same line carries:
   long_64k      chunkwise over 65536 tokens (1 x 16 heads)
   gated         the headline step with the output gate swish(G) (.) GN(o)
   backward      the chunkwise backward on the 1.3B-class layer
+  rotate        the xPos rotation of q and k of the 6.7B-class 8k layer, in
+                place; % of measured HBM
   cpu_baseline  the float64 CPU oracle on a bounded sample of the same
                 workload (rank 0, N = 1 only)
 With N > 1 (torchrun) every rank runs the same per-GPU step on its own GPU
@@ -596,6 +598,22 @@ def run_ours(args):
                              "tflops": Fb / cb / 1e12,
                              "note": "CUDA cores, float32; flops counted as twice the forward's"}
         del qb, kb, vb, dob, wsb
+        torch.cuda.empty_cache()
+
+        # ---------------- xPos rotation of q and k, 6.7B-class 8k layer ----------------
+        wr = wl.WORKLOADS["l6p7b_8k_bf16"]
+        qr, kr, vr, _ = make_qkv(torch, wr.B, wr.H, wr.N, wr.dk, wr.dv, device, seed=8000 + rank)
+        del vr
+        thr = torch.from_numpy(wl.rotation_angles(wr.dk, seed=1)).to(device)
+        tr, _ = timed(lambda: (ret.rotate(qr, thr, 0, out=qr), ret.rotate(kr, thr, 0, out=kr)),
+                      sub_steps, 3, stream, device)
+        launches += 2 * sub_steps
+        Br = 2 * 2 * qr.numel() * qr.element_size()   # q and k, each read and written once
+        cr = tr / sub_steps
+        extra["rotate"] = {"workload": "l6p7b_8k_bf16 xPos rotation of q and k, in place",
+                           "ms": cr * 1e3, "hbm_gbs": Br / cr / 1e9,
+                           "hbm_frac": Br / cr / 1e9 / peaks.get("hbm_gbs", 6650.0)}
+        del qr, kr
         torch.cuda.empty_cache()
 
         # ---------------- gated output on the headline workload ----------------

@@ -249,6 +249,31 @@ RET_API int ret_chunkwise_backward(const void* q, const void* k, const void* v,
                            int dk, int dv, int dtype, void* workspace, size_t workspace_bytes,
                            void* stream);
 
+/*
+ * xPos-style rotation of q or k rows ("RetNet - Retentive Network - A
+ * Successor to Transformer for LLMs", core components, item 3: a complex
+ * rotation that puts relative position into Q and K; "RetNet入門", Spiral.AI
+ * Tech Blog, LEX Transformer paragraph).  Channels (2c, 2c+1) of a row are
+ * the real and imaginary parts of one complex number, and the row at
+ * sequence position n is multiplied by e^{i n theta_c}:
+ *     y[2c]   = x[2c] cos(n theta_c) - x[2c+1] sin(n theta_c)
+ *     y[2c+1] = x[2c] sin(n theta_c) + x[2c+1] cos(n theta_c)
+ * Rotating both q and k makes q'_n . k'_m depend on n - m only.  The pages
+ * give neither the angles nor the channel pairing: theta is an input and the
+ * pairs are adjacent channels.
+ *   x     : [B][H][N][d] device, dtype, only read.
+ *   y     : [B][H][N][d] device, dtype, written; may equal x (in place), must
+ *           not overlap it otherwise.
+ *   theta : [d/2] float32 device array, radians per position for each pair.
+ *   pos0  : position of row 0 of every sequence (e.g. tokens already
+ *           decoded); 0 <= pos0 and pos0 + N <= 2^53.
+ * The angle n theta_c and its cos / sin are taken in double precision; the
+ * rotation itself in float32.  Supported: d even, N >= 0 (N == 0 writes
+ * nothing); x and y 16-byte aligned.
+ */
+RET_API int ret_rotate(const void* x, void* y, const float* theta, long long pos0, int B, int H,
+               int N, int d, int dtype, void* stream);
+
 /* Human-readable name of a ret_status value (static storage). */
 RET_API const char* ret_status_string(int status);
 

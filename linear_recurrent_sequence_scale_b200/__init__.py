@@ -42,6 +42,7 @@ SIGNATURES = {
     "ret_chunkwise_backward_workspace": (_S, [_I, _I, _I, _I, _I, _I, _I]),
     "ret_chunkwise_backward": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I,
                                     _I, _I, _I, _P, _S, _P]),
+    "ret_rotate": (_I, [_P, _P, _P, ctypes.c_longlong, _I, _I, _I, _I, _I, _P]),
     "ret_status_string": (ctypes.c_char_p, [_I]),
     "ret_last_cuda_error": (_I, []),
     "ret_version": (ctypes.c_char_p, []),
@@ -332,6 +333,31 @@ def state_combine(locals_, spans, r, gammas, state0=None, out=None):
                                          _ptr(out), B, H, dk, dv, _stream(dev))
     if s != RET_OK:
         _raise("ret_state_combine", s)
+    return out
+
+
+def rotate(x, theta, pos0=0, out=None):
+    """xPos-style rotation of q or k rows (ret_rotate): channel pair c of the
+    row at position pos0 + j turns by (pos0 + j) * theta[c].
+    x [B,H,N,d] or [B,H,d] (one position, e.g. a decode step); theta [d/2]
+    float32; out may be x itself (in place).  Returns out."""
+    torch = _torch()
+    if x.dim() not in (3, 4):
+        raise ValueError("x must be [B,H,N,d] or [B,H,d]")
+    B, H = x.shape[0], x.shape[1]
+    N = x.shape[2] if x.dim() == 4 else 1
+    d = x.shape[-1]
+    dev = x.device
+    _check(x, "x", device=dev)
+    code = _dtype_code(x)
+    _check(theta, "theta", dtype=torch.float32, shape=(d // 2,), device=dev)
+    if out is None:
+        out = torch.empty_like(x)
+    _check(out, "out", dtype=x.dtype, shape=tuple(x.shape), device=dev)
+    s = load_library().ret_rotate(_ptr(x), _ptr(out), _ptr(theta), int(pos0), B, H, N, d, code,
+                                  _stream(dev))
+    if s != RET_OK:
+        _raise("ret_rotate", s)
     return out
 
 

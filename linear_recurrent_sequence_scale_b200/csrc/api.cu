@@ -327,4 +327,20 @@ int ret_step(const void* q, const void* k, const void* v, const float* gammas, f
   return ret_step_gated(q, k, v, gammas, state, nullptr, o, B, H, dk, dv, dtype, gn_eps, stream);
 }
 
+int ret_rotate(const void* x, void* y, const float* theta, long long pos0, int B, int H, int N,
+               int d, int dtype, void* stream) {
+  if (B < 1 || H < 1 || N < 0 || d < 2 || d % 2) return RET_EINVAL;
+  if (!valid_dtype(dtype) || !x || !y || !theta) return RET_EINVAL;
+  if (pos0 < 0 || pos0 > ((long long)1 << 53) - N) return RET_EINVAL;
+  if (!aligned16(x) || !aligned16(y)) return RET_EINVAL;
+  if ((int64_t)B * H > INT32_MAX || (int64_t)N * d > ((int64_t)1 << 38) ||
+      (int64_t)B * H * N * d > ((int64_t)1 << 40))
+    return RET_EUNSUPPORTED;
+  const uintptr_t bytes = (uintptr_t)((int64_t)B * H * N * d * (dtype == RET_BF16 ? 2 : 4));
+  const uintptr_t xs = reinterpret_cast<uintptr_t>(x), ys = reinterpret_cast<uintptr_t>(y);
+  if (xs != ys && xs < ys + bytes && ys < xs + bytes) return RET_EINVAL;  // partial overlap
+  return cuda_status(ret::launch_rotate(x, y, theta, pos0, B, H, N, d, dtype,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

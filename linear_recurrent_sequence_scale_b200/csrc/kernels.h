@@ -38,6 +38,10 @@ cudaError_t launch_state_combine(const float* locals, const int* spans, int r,
                                  const float* gammas, const float* state0, float* out, int B,
                                  int H, int dk, int dv, cudaStream_t st);
 
+// xPos-style rotation of q or k rows by pos * theta per channel pair (rotate.cu).
+cudaError_t launch_rotate(const void* x, void* y, const float* theta, long long pos0, int B,
+                          int H, int N, int d, int dtype, cudaStream_t st);
+
 cudaError_t launch_simt_parallel(const void* q, const void* k, const void* v, const float* gammas,
                                  const void* gate, void* o, int B, int H, int N, int dk, int dv,
                                  int dtype, float eps, cudaStream_t st);

@@ -126,6 +126,14 @@ def make_inputs(B, H, N, dk, dv, dtype="bf16", seed=0, with_state=False, scale=N
     return {"q": q, "k": k, "v": v, "state": st, "gammas": g}
 
 
+def rotation_angles(d: int, seed: int = 0) -> np.ndarray:
+    """Angles (radians per position) for the d/2 channel pairs of the xPos
+    rotation: the pages give no values, so a geometric spread from 1 down to
+    1e-4, shuffled with the seed so that a mix-up of pairs changes the result."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return rng.permutation(np.geomspace(1.0, 1e-4, d // 2)).astype(np.float32)
+
+
 def make_head_inputs(w: Workload, b: int, h: int, N: int | None = None):
     """Inputs of one (batch, head) pair of a workload, drawn independently of
     the others, so that a sampled head can be rebuilt without drawing the

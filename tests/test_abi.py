@@ -207,3 +207,23 @@ def test_backward_rejects_bad_arguments(lib):
 def test_selftest_rejects_bad_limits(lib):
     assert lib.ret_selftest_bounded_wait(0, None) == ret.RET_EINVAL
     assert lib.ret_selftest_bounded_wait(20000, None) == ret.RET_EINVAL
+
+
+def test_rotate_rejects_bad_arguments(lib):
+    def call(x=A, y=A, th=A, pos0=0, B=1, H=2, N=300, d=64, dt=0):
+        return lib.ret_rotate(x, y, th, pos0, B, H, N, d, dt, None)
+
+    assert call(x=None) == ret.RET_EINVAL
+    assert call(y=None) == ret.RET_EINVAL
+    assert call(th=None) == ret.RET_EINVAL
+    assert call(x=M) == ret.RET_EINVAL
+    assert call(y=M) == ret.RET_EINVAL
+    assert call(d=63) == ret.RET_EINVAL
+    assert call(d=0) == ret.RET_EINVAL
+    assert call(N=-1) == ret.RET_EINVAL
+    assert call(B=0) == ret.RET_EINVAL
+    assert call(dt=5) == ret.RET_EINVAL
+    assert call(pos0=-1) == ret.RET_EINVAL
+    assert call(pos0=(1 << 53) - 299) == ret.RET_EINVAL
+    assert call(y=P(0x10000 + 64)) == ret.RET_EINVAL  # overlaps x without equalling it
+    assert call(N=0) == ret.RET_OK                   # nothing to launch

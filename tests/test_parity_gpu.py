@@ -528,3 +528,92 @@ def test_empty_sequence_copies_state(torch_cuda, ret):
     assert o.numel() == 0 and op.numel() == 0
     assert torch.equal(s, s0)
     assert torch.count_nonzero(z) == 0
+
+
+# --- xPos rotation ----------------------------------------------------------------
+
+def _rotation_close(y, ref, x_exact, dt):
+    """float32: 1e-5 rel-Frobenius.  bf16: one rounding of each output, so
+    |y - ref| <= 2^-8 |ref| + 1e-5 max|x| element by element."""
+    y = wl.from_torch(y)
+    if dt == "f32":
+        assert oracle.rel_frobenius(y, ref) < TOL["f32"]
+    else:
+        bound = 2.0 ** -8 * np.abs(ref) + 1e-5 * np.max(np.abs(x_exact))
+        assert np.all(np.abs(y - ref) <= bound)
+
+
+# (dtype, B, H, N, d, pos0): d % 8 != 0 takes the one-pair-per-thread path;
+# B*H = 17 and 5 leave partial 4-row groups and 16-row shares; a pos0 of 1.2e8
+# turns pairs by up to 1.2e8 rad.
+ROT_CASES = [("f32", 2, 3, 300, 64, 0), ("bf16", 2, 3, 300, 64, 5), ("f32", 1, 2, 37, 6, 0),
+             ("bf16", 1, 2, 129, 10, 1000000), ("f32", 1, 5, 17, 256, 123456789),
+             ("bf16", 1, 17, 64, 512, 7), ("bf16", 4, 16, 70, 128, 3)]
+
+
+@pytest.mark.parametrize("case", ROT_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_rotate_parity(torch_cuda, ret, case):
+    torch = torch_cuda
+    dt, B, H, N, d, pos0 = case
+    rng = np.random.Generator(np.random.PCG64(N * 131 + d))
+    x = wl.draw(rng, (B, H, N, d), 1.0, dt)
+    th = wl.rotation_angles(d, seed=d)
+    ref = oracle.rotate(x.exact, th.astype(np.float64), pos0)
+    xd = _dev(x)
+    y = ret.rotate(xd, torch.from_numpy(th).cuda(), pos0)
+    _rotation_close(y, ref, x.exact, dt)
+    ret.rotate(xd, torch.from_numpy(th).cuda(), pos0, out=xd)   # in place
+    torch.cuda.synchronize()
+    assert torch.equal(xd, y)
+
+
+def test_rotate_decode_row_and_empty(torch_cuda, ret):
+    """One position per (batch, head), as in a decode step at position 4095;
+    an empty sequence writes nothing."""
+    torch = torch_cuda
+    rng = np.random.Generator(np.random.PCG64(77))
+    x = wl.draw(rng, (2, 4, 256), 1.0, "bf16")
+    th = wl.rotation_angles(256, seed=3)
+    y = ret.rotate(_dev(x), torch.from_numpy(th).cuda(), 4095)
+    ref = oracle.rotate(x.exact[:, :, None, :], th.astype(np.float64), 4095)[:, :, 0]
+    _rotation_close(y, ref, x.exact, "bf16")
+    e = torch.full((1, 2, 0, 64), 3.0, device="cuda")
+    assert ret.rotate(e, torch.from_numpy(wl.rotation_angles(64)).cuda()).shape == e.shape
+
+
+def test_rotated_retention_matches_oracle(torch_cuda, ret):
+    """Rotation followed by retention (parallel and chunkwise) against the
+    oracle's rotation followed by its recurrence."""
+    torch = torch_cuda
+    inp = wl.make_inputs(1, 2, 96, 16, 8, "f32", seed=41)
+    th = wl.rotation_angles(16, seed=5)
+    tht = torch.from_numpy(th).cuda()
+    qr = ret.rotate(_dev(inp["q"]), tht, 11)
+    kr = ret.rotate(_dev(inp["k"]), tht, 11)
+    g = _gam(torch, inp["gammas"])
+    o_ref, _ = oracle.recurrent(oracle.rotate(inp["q"].exact, th.astype(np.float64), 11),
+                                oracle.rotate(inp["k"].exact, th.astype(np.float64), 11),
+                                inp["v"].exact, inp["gammas"])
+    v = _dev(inp["v"])
+    assert _rel(ret.parallel(qr, kr, v, g), o_ref) < TOL["f32"]
+    assert _rel(ret.chunkwise(qr, kr, v, g, 32), o_ref) < TOL["f32"]
+
+
+def test_rotate_full_size_sampled(torch_cuda, ret):
+    """The 6.7B-class 8k layer's q (8 x 16 x 8192 x 256, bf16) rotated in
+    place as the bench does; sampled rows against the oracle."""
+    torch = torch_cuda
+    B, H, N, d = 8, 16, 8192, 256
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    x = torch.randn((B, H, N, d), device="cuda", generator=gen).bfloat16()
+    th = wl.rotation_angles(d, seed=9)
+    rows = [(0, 0, 0), (7, 15, 8191), (3, 9, 4097), (5, 2, 1), (1, 14, 6000)]
+    before = [wl.from_torch(x[b, h, n]) for b, h, n in rows]
+    ret.rotate(x, torch.from_numpy(th).cuda(), 0, out=x)
+    torch.cuda.synchronize()
+    for (b, h, n), xe in zip(rows, before):
+        ref = oracle.rotate(xe[None, :], th.astype(np.float64), n)[0]
+        _rotation_close(x[b, h, n], ref, xe, "bf16")
+    del x
+    torch.cuda.empty_cache()
