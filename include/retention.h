@@ -269,7 +269,7 @@ RET_API int ret_chunkwise_backward(const void* q, const void* k, const void* v,
  *           decoded); 0 <= pos0 and pos0 + N <= 2^53.
  * The angle n theta_c and its cos / sin are taken in double precision; the
  * rotation itself in float32.  Supported: d even, N >= 0 (N == 0 writes
- * nothing); x and y 16-byte aligned.
+ * nothing, and x, y and theta may then be NULL); x and y 16-byte aligned.
  */
 RET_API int ret_rotate(const void* x, void* y, const float* theta, long long pos0, int B, int H,
                int N, int d, int dtype, void* stream);

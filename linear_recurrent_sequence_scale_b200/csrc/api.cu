@@ -330,8 +330,10 @@ int ret_step(const void* q, const void* k, const void* v, const float* gammas, f
 int ret_rotate(const void* x, void* y, const float* theta, long long pos0, int B, int H, int N,
                int d, int dtype, void* stream) {
   if (B < 1 || H < 1 || N < 0 || d < 2 || d % 2) return RET_EINVAL;
-  if (!valid_dtype(dtype) || !x || !y || !theta) return RET_EINVAL;
+  if (!valid_dtype(dtype)) return RET_EINVAL;
   if (pos0 < 0 || pos0 > ((long long)1 << 53) - N) return RET_EINVAL;
+  if (N == 0) return RET_OK;  // nothing to read or write; x, y, theta may be NULL
+  if (!x || !y || !theta) return RET_EINVAL;
   if (!aligned16(x) || !aligned16(y)) return RET_EINVAL;
   if ((int64_t)B * H > INT32_MAX || (int64_t)N * d > ((int64_t)1 << 38) ||
       (int64_t)B * H * N * d > ((int64_t)1 << 40))

@@ -227,3 +227,4 @@ def test_rotate_rejects_bad_arguments(lib):
     assert call(pos0=(1 << 53) - 299) == ret.RET_EINVAL
     assert call(y=P(0x10000 + 64)) == ret.RET_EINVAL  # overlaps x without equalling it
     assert call(N=0) == ret.RET_OK                   # nothing to launch
+    assert call(N=0, x=None, y=None, th=None) == ret.RET_OK
