@@ -236,7 +236,10 @@ RET_API int ret_state_combine(const float* locals, const int* spans, int r, cons
  *   state_in     : the forward call's initial state, or NULL (zero)
  *   d_state_out  : [B][H][dk][dv] float32, or NULL (zero)
  *   workspace    : at least ret_chunkwise_backward_workspace() bytes; holds
- *                  the forward and the gradient chunk states in float32.
+ *                  the forward and the gradient chunk states and the masked
+ *                  in-chunk scores, all float32, for chunks of
+ *                  min(chunk, 128) tokens (the gradients do not depend on
+ *                  the chunk length).
  * Runs on the CUDA cores in float32 for either dtype and any chunk >= 1,
  * dk, dv in [8, 512].  Errors as for ret_chunkwise.
  */

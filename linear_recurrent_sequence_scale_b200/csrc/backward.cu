@@ -14,9 +14,9 @@
 // and the gradient of the incoming state is G_{-1}.
 //   1. the forward chunk states R_{i-1} (the chunkwise states phase, float32)
 //   2. grad_scan: G_i for every chunk, walking the chunks backwards
-//   3. chunk_grad: per (b, h, chunk, 16 positions) the in-chunk parts of the
-//      three row gradients
-//   4. cross_chunk_gemm: the cross-chunk parts, one batched GEMM each.
+//   3. chunk_scores: D (.) (dO V^T) and D (.) (Q K^T) per chunk, float32
+//   4. chunk_grads: dQ, dK, dV, each one batched product per chunk that adds
+//      the cross-chunk term to the in-chunk one.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -25,8 +25,6 @@ namespace bwd {
 
 constexpr int ST = 64;  // state tile edge of the scan
 constexpr int SJ = 32;  // tokens staged per scan step
-constexpr int TP = 16;  // positions per gradient tile
-constexpr int MAXU = 32;  // columns per thread: d <= 16 * MAXU = 512
 
 // G_i = gradient of the state leaving chunk i, for i = nc-1 down to 0, into
 // gws slot i; the gradient of the incoming state at the end.
@@ -110,249 +108,212 @@ grad_scan(const T* __restrict__ q, const T* __restrict__ dout, const float* __re
   }
 }
 
-// Rows [n, n + rows) of a [.., N, d] tensor of (b, h) into smem with row
-// stride ld (zeros past `rows`).
-template <typename T>
-__device__ __forceinline__ void stage_rows(float* dst, int ld, const T* src, int bh, int N, int d,
-                                           int n, int rows) {
-  for (int e = threadIdx.x; e < TP * d; e += 256) {
-    const int r = e / d, x = e % d;
-    dst[r * ld + x] = r < rows ? Elem<T>::ld(src + ((size_t)bh * N + n + r) * d + x) : 0.f;
-  }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(256)
-chunk_grad(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-           const T* __restrict__ dout, const float* __restrict__ gammas, int chunk,
-           T* __restrict__ dq, T* __restrict__ dk_, T* __restrict__ dv_, int H, int N, int dk,
-           int dv) {
-  extern __shared__ float sm[];
-  const int lk = dk + 1, lv = dv + 1;
-  float* a_v = sm;                 // [TP][dv+1]  tile rows: dO (phase A) / V (phase B)
-  float* a_k = a_v + TP * lv;      // [TP][dk+1]  tile rows: K (phase B)
-  float* b_v = a_k + TP * lk;      // [TP][dv+1]  other rows: V (A) / dO (B)
-  float* b_k = b_v + TP * lv;      // [TP][dk+1]  other rows: K (A) / Q (B)
-  float* ps = b_k + TP * lk;       // [TP][TP+1]
-  float* ss = ps + TP * (TP + 1);  // [TP][TP+1]
-
-  const int bh = blockIdx.y;
-  const float lg = log2f(gammas[bh % H]);
-  const int tpc = cdiv(chunk, TP);
-  const int ci = blockIdx.x / tpc;
-  const int cs = ci * chunk;
-  const int p0 = cs + (blockIdx.x % tpc) * TP;
-  const int ce = min(N, cs + chunk);
-  if (p0 >= ce) return;
-  const int rows = min(TP, ce - p0);
-  const int tid = threadIdx.x;
-  const int t = tid & 15, cg = tid >> 4;  // accumulation: row t, columns cg + 16 x
-  const int da = tid >> 4, db = tid & 15;  // dot products: pair (da, db)
-
-  // ---- phase A: dQ rows of this tile ----
-  float acc[MAXU];
-#pragma unroll
-  for (int x = 0; x < MAXU; ++x) acc[x] = 0.f;
-  stage_rows(a_v, lv, dout, bh, N, dv, p0, rows);
-  for (int m0 = cs; m0 < p0 + rows; m0 += TP) {
-    const int mr = min(TP, p0 + rows - m0);
-    __syncthreads();
-    stage_rows(b_v, lv, v, bh, N, dv, m0, mr);
-    stage_rows(b_k, lk, k, bh, N, dk, m0, mr);
-    __syncthreads();
-    {  // ps[n][m] = D_nm (dO_n . v_m)
-      float s = 0.f;
-      for (int j = 0; j < dv; ++j) s = fmaf(a_v[da * lv + j], b_v[db * lv + j], s);
-      const int n = p0 + da, m = m0 + db;
-      ps[da * (TP + 1) + db] = (da < rows && db < mr && m <= n) ? s * gpow(lg, n - m) : 0.f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int x = 0; x < MAXU; ++x) {
-      const int c = cg + 16 * x;
-      if (c < dk) {
-        float s = acc[x];
-        for (int b = 0; b < TP; ++b) s = fmaf(ps[t * (TP + 1) + b], b_k[b * lk + c], s);
-        acc[x] = s;
-      }
-    }
-  }
-  if (t < rows) {
-    const int n = p0 + t;
-#pragma unroll
-    for (int x = 0; x < MAXU; ++x) {
-      const int c = cg + 16 * x;
-      if (c < dk) Elem<T>::st(dq + ((size_t)bh * N + n) * dk + c, acc[x]);
-    }
-  }
-
-  // ---- phase B: dK and dV rows of this tile ----
-  float acck[MAXU], accv[MAXU];
-#pragma unroll
-  for (int x = 0; x < MAXU; ++x) acck[x] = accv[x] = 0.f;
-  __syncthreads();
-  stage_rows(a_v, lv, v, bh, N, dv, p0, rows);
-  stage_rows(a_k, lk, k, bh, N, dk, p0, rows);
-  for (int n0 = p0; n0 < ce; n0 += TP) {
-    const int nr = min(TP, ce - n0);
-    __syncthreads();
-    stage_rows(b_v, lv, dout, bh, N, dv, n0, nr);
-    stage_rows(b_k, lk, q, bh, N, dk, n0, nr);
-    __syncthreads();
-    {  // ps[n][m] = D_nm (dO_n . v_m), ss[n][m] = D_nm (q_n . k_m)
-      float sp = 0.f, sq = 0.f;
-      for (int j = 0; j < dv; ++j) sp = fmaf(b_v[da * lv + j], a_v[db * lv + j], sp);
-      for (int j = 0; j < dk; ++j) sq = fmaf(b_k[da * lk + j], a_k[db * lk + j], sq);
-      const int n = n0 + da, m = p0 + db;
-      const float w = (da < nr && db < rows && n >= m) ? gpow(lg, n - m) : 0.f;
-      ps[da * (TP + 1) + db] = sp * w;
-      ss[da * (TP + 1) + db] = sq * w;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int x = 0; x < MAXU; ++x) {
-      const int c = cg + 16 * x;
-      if (c < dk) {
-        float s = acck[x];
-        for (int a = 0; a < TP; ++a) s = fmaf(ps[a * (TP + 1) + t], b_k[a * lk + c], s);
-        acck[x] = s;
-      }
-      if (c < dv) {
-        float s = accv[x];
-        for (int a = 0; a < TP; ++a) s = fmaf(ss[a * (TP + 1) + t], b_v[a * lv + c], s);
-        accv[x] = s;
-      }
-    }
-  }
-  if (t < rows) {
-    const int m = p0 + t;
-#pragma unroll
-    for (int x = 0; x < MAXU; ++x) {
-      const int c = cg + 16 * x;
-      if (c < dk) Elem<T>::st(dk_ + ((size_t)bh * N + m) * dk + c, acck[x]);
-      if (c < dv) Elem<T>::st(dv_ + ((size_t)bh * N + m) * dv + c, accv[x]);
-    }
-  }
-}
-
-// Cross-chunk terms as one batched GEMM per (b, h, chunk), added to the
-// rows chunk_grad wrote:
-//     out[n] += s_n * (A[n] . S')    over the chunk's positions n,
-// with S' = S^T (TRANS: dQ += xi (.) dO R_{i-1}^T, dK += zeta (.) V G_i^T) or
-// S' = S (dV += zeta (.) K G_i), S a float32 [dk][dv] chunk state.  Tiles of
-// 64 rows x 64 columns, 4 x 4 results per thread, 16-deep slices of A and S'
-// through shared memory.
+// ---- register-tiled products: 64 x 64 results per CTA, 4 x 4 per thread,
+// 16-deep slices of both operands through shared memory ----
 constexpr int GM = 64, GN_ = 64, GK = 16;
 
-template <typename T, bool TRANS, bool XI>
-__global__ void __launch_bounds__(256)
-cross_chunk_gemm(const T* __restrict__ a, const float* __restrict__ states, int has_r0,
-                 const float* __restrict__ gammas, int chunk, T* __restrict__ out, int H, int N,
-                 int ka, int ncol, int dk, int dv) {
-  __shared__ float as[GK][GM + 4];
-  __shared__ float bs[GK][GN_ + 4];
-  const int nc = cdiv(N, chunk);
-  const int rpc = cdiv(chunk, GM);        // row blocks per chunk
-  const int ci = blockIdx.y / rpc;
-  const int cs = ci * chunk;
-  const int r0 = cs + (blockIdx.y % rpc) * GM;
-  const int ce = min(N, cs + chunk);
-  if (r0 >= ce || (XI && ci == 0 && !has_r0)) return;
-  const int bh = blockIdx.z;
-  const int c0 = blockIdx.x * GN_;
-  const float lg = log2f(gammas[bh % H]);
-  const float* S = states + ((size_t)bh * nc + ci) * dk * dv;
+struct Tile {
+  float as[GK][GM + 4];
+  float bs[GK][GN_ + 4];
+};
+
+// acc += A[.., k0 .. k1) B[k0 .. k1), ..] over this CTA's 64 x 64 tile, with
+// la(r, k) = A[r][k] and lb(k, c) = B[k][c] (tile-local r, c; both return 0
+// outside the operand).  A_KC / B_KC: consecutive k of one r (of one c) are
+// adjacent in memory, so consecutive threads load along k; otherwise they
+// load along r (along c).
+template <bool A_KC, bool B_KC, class LA, class LB>
+__device__ __forceinline__ void tile_product(Tile& t, LA la, LB lb, int k0, int k1,
+                                             float (&acc)[4][4]) {
   const int tid = threadIdx.x;
   const int ty = tid >> 4, tx = tid & 15;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < ka; k0 += GK) {
+  for (int kb = k0; kb < k1; kb += GK) {
     __syncthreads();
-    for (int e = tid; e < GM * GK; e += 256) {  // A rows r0.., columns k0..
-      const int r = e / GK, kk = e % GK;
-      const int n = r0 + r;
-      as[kk][r] = (n < ce && k0 + kk < ka) ? Elem<T>::ld(a + ((size_t)bh * N + n) * ka + k0 + kk)
-                                           : 0.f;
+    for (int e = tid; e < GM * GK; e += 256) {
+      const int r = A_KC ? e / GK : e % GM;
+      const int kk = A_KC ? e % GK : e / GM;
+      t.as[kk][r] = kb + kk < k1 ? la(r, kb + kk) : 0.f;
     }
-    for (int e = tid; e < GK * GN_; e += 256) {  // S' rows k0.., columns c0..
-      int kk, c;
-      if (TRANS) { c = e / GK; kk = e % GK; } else { kk = e / GN_; c = e % GN_; }
-      float x = 0.f;
-      if (k0 + kk < ka && c0 + c < ncol)
-        x = TRANS ? S[(size_t)(c0 + c) * dv + k0 + kk] : S[(size_t)(k0 + kk) * dv + c0 + c];
-      bs[kk][c] = x;
+    for (int e = tid; e < GK * GN_; e += 256) {
+      const int c = B_KC ? e / GK : e % GN_;
+      const int kk = B_KC ? e % GK : e / GN_;
+      t.bs[kk][c] = kb + kk < k1 ? lb(kb + kk, c) : 0.f;
     }
     __syncthreads();
 #pragma unroll
     for (int kk = 0; kk < GK; ++kk) {
       float av[4], bv[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) av[i] = as[kk][ty * 4 + i];
+      for (int i = 0; i < 4; ++i) av[i] = t.as[kk][ty * 4 + i];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) bv[j] = bs[kk][tx * 4 + j];
+      for (int j = 0; j < 4; ++j) bv[j] = t.bs[kk][tx * 4 + j];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
   }
-  const int L = ce - cs;
+}
+
+// Masked scores of one chunk, S[n][m] = D_nm (x_n . y_m) for in-chunk
+// positions n, m < L, into a float32 [chunk][chunk] slot per (b, h, chunk):
+// P = D (.) (dO V^T) for dQ and dK, and D (.) (Q K^T) for dV.  Only tiles
+// on or below the diagonal are computed; nothing reads the others.
+// Grid: x = chunk, y = lower-triangular tile pair, z = (b, h).
+template <typename T>
+__global__ void __launch_bounds__(256)
+chunk_scores(const T* __restrict__ x, const T* __restrict__ y, const float* __restrict__ gammas,
+             int chunk, float* __restrict__ out, int H, int N, int d) {
+  __shared__ Tile t;
+  int i = 0;
+  while ((i + 1) * (i + 2) / 2 <= (int)blockIdx.y) ++i;
+  const int j = blockIdx.y - i * (i + 1) / 2;  // row tile i >= column tile j
+  const int ci = blockIdx.x, bh = blockIdx.z;
+  const int cs = ci * chunk;
+  const int L = min(chunk, N - cs);
+  const int r0 = i * GM, c0 = j * GN_;
+  if (r0 >= L) return;
+  const T* X = x + ((size_t)bh * N + cs) * d;
+  const T* Y = y + ((size_t)bh * N + cs) * d;
+  float acc[4][4] = {};
+  tile_product<true, true>(
+      t,
+      [&](int r, int k) { return r0 + r < L ? Elem<T>::ld(X + (size_t)(r0 + r) * d + k) : 0.f; },
+      [&](int k, int c) { return c0 + c < L ? Elem<T>::ld(Y + (size_t)(c0 + c) * d + k) : 0.f; },
+      0, d, acc);
+  const float lg = log2f(gammas[bh % H]);
+  float* S = out + ((size_t)bh * gridDim.x + ci) * chunk * chunk;
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int n = r0 + ty * 4 + i;
-    if (n >= ce) continue;
-    const float sc = XI ? gpow(lg, n - cs + 1) : gpow(lg, L - 1 - (n - cs));
-    T* orow = out + ((size_t)bh * N + n) * ncol;
+  for (int a = 0; a < 4; ++a) {
+    const int n = r0 + ty * 4 + a;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = c0 + tx * 4 + j;
-      if (c < ncol) Elem<T>::st(orow + c, Elem<T>::ld(orow + c) + sc * acc[i][j]);
+    for (int b = 0; b < 4; ++b) {
+      const int m = c0 + tx * 4 + b;
+      if (n < L && m < L) S[(size_t)n * chunk + m] = m <= n ? gpow(lg, n - m) * acc[a][b] : 0.f;
     }
   }
 }
+
+// One gradient of one chunk, the in-chunk and the cross-chunk product in one
+// accumulation (positions n, m in the chunk, P and S the scores above,
+// R = R_{i-1}, G = G_i, both float32 [dk][dv]):
+//   MODE 0  dQ[n] = sum_{m<=n} P[n][m] k_m + xi_n   (dO_n R^T)
+//   MODE 1  dK[m] = sum_{n>=m} P[n][m] q_n + zeta_m (v_m G^T)
+//   MODE 2  dV[m] = sum_{n>=m} S[n][m] dO_n + zeta_m (k_m G)
+// b1 holds the rows the scores multiply (k, q, dO), a2 those the state
+// multiplies (dO, v, k; a2 rows are d2 wide), out is ncol wide.  Grid: x =
+// chunk, y = (64-row tile, 64-column tile), z = (b, h).
+template <typename T, int MODE>
+__global__ void __launch_bounds__(256)
+chunk_grads(const T* __restrict__ b1, const T* __restrict__ a2, const float* __restrict__ scores,
+            const float* __restrict__ states, int has_r0, const float* __restrict__ gammas,
+            int chunk, T* __restrict__ out, int H, int N, int d2, int ncol, int dk, int dv) {
+  __shared__ Tile t;
+  __shared__ float rsc[GM];
+  const int ctn = cdiv(ncol, GN_);
+  const int r0 = (blockIdx.y / ctn) * GM, c0 = (blockIdx.y % ctn) * GN_;
+  const int ci = blockIdx.x, bh = blockIdx.z;
+  const int cs = ci * chunk;
+  const int L = min(chunk, N - cs);
+  if (r0 >= L) return;
+  const float* P = scores + ((size_t)bh * gridDim.x + ci) * chunk * chunk;
+  const T* B1 = b1 + ((size_t)bh * N + cs) * ncol;
+  float acc[4][4] = {};
+  if (MODE == 0)
+    tile_product<true, false>(
+        t, [&](int r, int k) { return r0 + r < L ? P[(size_t)(r0 + r) * chunk + k] : 0.f; },
+        [&](int k, int c) { return c0 + c < ncol ? Elem<T>::ld(B1 + (size_t)k * ncol + c0 + c) : 0.f; },
+        0, min(L, r0 + GM), acc);
+  else
+    tile_product<false, false>(
+        t, [&](int r, int k) { return r0 + r < L ? P[(size_t)k * chunk + r0 + r] : 0.f; },
+        [&](int k, int c) { return c0 + c < ncol ? Elem<T>::ld(B1 + (size_t)k * ncol + c0 + c) : 0.f; },
+        r0, L, acc);
+  if (MODE != 0 || ci > 0 || has_r0) {
+    const float lg = log2f(gammas[bh % H]);
+    if (threadIdx.x < GM) {
+      const int jj = r0 + threadIdx.x;  // xi_j = gamma^(j+1), zeta_j = gamma^(L-1-j)
+      rsc[threadIdx.x] = jj < L ? gpow(lg, MODE == 0 ? jj + 1 : L - 1 - jj) : 0.f;
+    }
+    const float* St = states + ((size_t)bh * gridDim.x + ci) * dk * dv;
+    const T* A2 = a2 + ((size_t)bh * N + cs) * d2;
+    auto la = [&](int r, int k) {
+      return r0 + r < L ? rsc[r] * Elem<T>::ld(A2 + (size_t)(r0 + r) * d2 + k) : 0.f;
+    };
+    // rsc is written before the first barrier inside tile_product
+    if (MODE == 2)
+      tile_product<true, false>(
+          t, la, [&](int k, int c) { return c0 + c < ncol ? St[(size_t)k * dv + c0 + c] : 0.f; },
+          0, d2, acc);
+    else
+      tile_product<true, true>(
+          t, la, [&](int k, int c) { return c0 + c < ncol ? St[(size_t)(c0 + c) * dv + k] : 0.f; },
+          0, d2, acc);
+  }
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int n = r0 + ty * 4 + a;
+    if (n >= L) continue;
+    T* orow = out + ((size_t)bh * N + cs + n) * ncol;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int c = c0 + tx * 4 + b;
+      if (c < ncol) Elem<T>::st(orow + c, acc[a][b]);
+    }
+  }
+}
+
+// The chunk length the backward works in.  Every chunk length gives the same
+// forward output in exact arithmetic, so the gradients do not depend on it;
+// 128 keeps both the [chunk][chunk] scores and the per-chunk states small.
+inline int work_chunk(int chunk) { return chunk < 128 ? chunk : 128; }
 
 template <typename T>
 cudaError_t backward_t(const void* q, const void* k, const void* v, const float* gammas, int chunk,
                        const float* state_in, const void* dout, const float* d_state_out,
                        void* dq, void* dk_, void* dv_, float* d_state_in, int B, int H, int N,
                        int dk, int dv, int dtype, void* ws, cudaStream_t st) {
+  chunk = work_chunk(chunk);
   const int nc = cdiv(N, chunk);
+  const size_t slots = (size_t)B * H * nc;
   float* rws = static_cast<float*>(ws);
-  float* gws = rws + (size_t)B * H * nc * dk * dv;
+  float* gws = rws + slots * dk * dv;
+  float* pws = gws + slots * dk * dv;
+  float* sws = pws + slots * chunk * chunk;
   cudaError_t e = launch_simt_states(k, v, gammas, chunk, state_in, nullptr, B, H, N, dk, dv,
                                      dtype, rws, st);
   if (e != cudaSuccess) return e;
+  const T* Q = static_cast<const T*>(q);
+  const T* K = static_cast<const T*>(k);
+  const T* V = static_cast<const T*>(v);
+  const T* dO = static_cast<const T*>(dout);
   dim3 g1(cdiv(dv, ST), cdiv(dk, ST), B * H);
-  grad_scan<T><<<g1, 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(dout), gammas,
-                                   chunk, d_state_out, d_state_in, gws, H, N, dk, dv);
+  grad_scan<T><<<g1, 256, 0, st>>>(Q, dO, gammas, chunk, d_state_out, d_state_in, gws, H, N, dk,
+                                   dv);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-  const size_t smem =
-      sizeof(float) * (size_t)(2 * TP * (dv + 1) + 2 * TP * (dk + 1) + 2 * TP * (TP + 1));
-  auto fn = chunk_grad<T>;
-  if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-      cudaSuccess)
-    return e;
-  dim3 g2(nc * cdiv(chunk, TP), B * H);
-  fn<<<g2, 256, smem, st>>>(static_cast<const T*>(q), static_cast<const T*>(k),
-                            static_cast<const T*>(v), static_cast<const T*>(dout), gammas, chunk,
-                            static_cast<T*>(dq),
-                            static_cast<T*>(dk_), static_cast<T*>(dv_), H, N, dk, dv);
+  const int nt = cdiv(chunk, GM);
+  const dim3 gs(nc, nt * (nt + 1) / 2, B * H);
+  chunk_scores<T><<<gs, 256, 0, st>>>(dO, V, gammas, chunk, pws, H, N, dv);
+  chunk_scores<T><<<gs, 256, 0, st>>>(Q, K, gammas, chunk, sws, H, N, dk);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
-  const int rb = nc * cdiv(chunk, GM);
-  const dim3 gq(cdiv(dk, GN_), rb, B * H), gv_(cdiv(dv, GN_), rb, B * H);
-  cross_chunk_gemm<T, true, true><<<gq, 256, 0, st>>>(
-      static_cast<const T*>(dout), rws, state_in != nullptr, gammas, chunk, static_cast<T*>(dq), H,
-      N, dv, dk, dk, dv);
-  cross_chunk_gemm<T, true, false><<<gq, 256, 0, st>>>(
-      static_cast<const T*>(v), gws, 1, gammas, chunk, static_cast<T*>(dk_), H, N, dv, dk, dk, dv);
-  cross_chunk_gemm<T, false, false><<<gv_, 256, 0, st>>>(
-      static_cast<const T*>(k), gws, 1, gammas, chunk, static_cast<T*>(dv_), H, N, dk, dv, dk, dv);
+  const dim3 gk(nc, nt * cdiv(dk, GN_), B * H), gv(nc, nt * cdiv(dv, GN_), B * H);
+  const int r0 = state_in != nullptr;
+  chunk_grads<T, 0><<<gk, 256, 0, st>>>(K, dO, pws, rws, r0, gammas, chunk, static_cast<T*>(dq),
+                                        H, N, dv, dk, dk, dv);
+  chunk_grads<T, 1><<<gk, 256, 0, st>>>(Q, V, pws, gws, 1, gammas, chunk, static_cast<T*>(dk_), H,
+                                        N, dv, dk, dk, dv);
+  chunk_grads<T, 2><<<gv, 256, 0, st>>>(dO, K, sws, gws, 1, gammas, chunk, static_cast<T*>(dv_), H,
+                                        N, dk, dv, dk, dv);
   return cudaPeekAtLastError();
 }
 
 }  // namespace bwd
 
 size_t backward_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk) {
-  return 2 * sizeof(float) * (size_t)B * H * cdiv(N, chunk) * dk * dv;
+  const int c = bwd::work_chunk(chunk);
+  return 2 * sizeof(float) * (size_t)B * H * cdiv(N, c) * ((size_t)dk * dv + (size_t)c * c);
 }
 
 cudaError_t launch_chunkwise_backward(const void* q, const void* k, const void* v,

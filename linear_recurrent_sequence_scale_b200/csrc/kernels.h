@@ -23,7 +23,7 @@ cudaError_t launch_simt_output(const void* q, const void* k, const void* v, cons
                                int dv, int dtype, float eps, const void* ws, cudaStream_t st);
 
 // Chunkwise backward on the CUDA cores (backward.cu); ws holds the forward
-// and the gradient chunk states in float32.
+// and the gradient chunk states and the in-chunk scores in float32.
 size_t backward_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk);
 cudaError_t launch_chunkwise_backward(const void* q, const void* k, const void* v,
                                       const float* gammas, int chunk, const float* state_in,
