@@ -186,6 +186,12 @@ def test_state_combine_rejects_bad_arguments(lib):
 def test_backward_rejects_bad_arguments(lib):
     need = lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 64, 64, 0)
     assert need > 0 and lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 64, 0, 0) == 0
+    # float32 forward and gradient states plus two [c][c] score blocks per chunk of
+    # c = min(chunk, 128) tokens
+    for chunk, c in ((64, 64), (37, 37), (512, 128)):
+        nc = -(-300 // c)
+        assert lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 96, chunk, 1) == \
+            2 * 4 * 2 * nc * (64 * 96 + c * c)
 
     def call(q=A, dO=A, gq=A, ds=A, si=None, dso=None, ws=A, wsb=None, N=300, chunk=64, dt=0):
         wsb = need if wsb is None else wsb
