@@ -590,7 +590,7 @@ def run_ours(args):
             device=device)
         tb, _ = timed(lambda: ret.chunkwise_backward(qb, kb, vb, gb, wb.chunk, dob, workspace=wsb),
                       3, 1, stream, device)
-        launches += 3 * 7
+        launches += 3 * 7   # two state scans, two score and three gradient products
         Fb = 2 * chunkwise_flops(wb.B, wb.H, wb.N, wb.dk, wb.dv, wb.chunk)
         cb = tb / 3
         extra["backward"] = {"workload": "l1p3b_bf16 chunkwise backward (dq, dk, dv)",

@@ -12,8 +12,8 @@
 //     dK_[i]    = (dO V^T (.) D)^T Q + zeta (.) (V G_i^T)
 //     dV_[i]    = (Q K^T (.) D)^T dO + zeta (.) (K G_i)
 // and the gradient of the incoming state is G_{-1}.
-//   1. the forward chunk states R_{i-1} (the chunkwise states phase, float32)
-//   2. grad_scan: G_i for every chunk, walking the chunks backwards
+//   1. state_scan<FWD>: the forward chunk states R_{i-1}, float32
+//   2. state_scan<!FWD>: G_i for every chunk, walking the chunks backwards
 //   3. chunk_scores: D (.) (dO V^T) and D (.) (Q K^T) per chunk, float32
 //   4. chunk_grads: dQ, dK, dV, each one batched product per chunk that adds
 //      the cross-chunk term to the in-chunk one.
@@ -26,15 +26,22 @@ namespace bwd {
 constexpr int ST = 64;  // state tile edge of the scan
 constexpr int SJ = 32;  // tokens staged per scan step
 
-// G_i = gradient of the state leaving chunk i, for i = nc-1 down to 0, into
-// gws slot i; the gradient of the incoming state at the end.
-template <typename T>
-__global__ void __launch_bounds__(256)
-grad_scan(const T* __restrict__ q, const T* __restrict__ dout, const float* __restrict__ gammas,
-          int chunk, const float* __restrict__ d_state_out, float* __restrict__ d_state_in,
-          float* __restrict__ gws, int H, int N, int dk, int dv) {
-  __shared__ float qs[SJ][ST];
-  __shared__ float ds[SJ][ST];
+// The two chunk-state recurrences of the backward, one 64 x 64 tile of the
+// d_k x d_v state per CTA, walking the chunks in order:
+//   FWD    slot i = R_{i-1} (the state entering chunk i), starting from
+//          state_in:   R_i = gamma^L R_{i-1} + K_[i]^T (V_[i] (.) zeta)
+//   !FWD   slot i = G_i (the gradient of the state leaving chunk i), from
+//          the last chunk down, starting from d_state_out:
+//          G_{i-1} = gamma^L G_i + (Q_[i] (.) xi)^T dO_[i];  G_{-1} is written
+//          to `last` (the gradient of state_in) when it is not null.
+// a is K (FWD) or Q, [.., N, dk]; b is V (FWD) or dO, [.., N, dv].
+template <typename T, bool FWD>
+__global__ void __launch_bounds__(256, 4)
+state_scan(const T* __restrict__ a, const T* __restrict__ b, const float* __restrict__ gammas,
+           int chunk, const float* __restrict__ first, float* __restrict__ last,
+           float* __restrict__ slots, int H, int N, int dk, int dv) {
+  __shared__ float as[SJ][ST];
+  __shared__ float bs[SJ][ST];
   const int bh = blockIdx.z;
   const float lg = log2f(gammas[bh % H]);
   const int r0 = blockIdx.y * ST;
@@ -49,17 +56,17 @@ grad_scan(const T* __restrict__ q, const T* __restrict__ dout, const float* __re
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int r = r0 + ty * 4 + i, c = c0 + tx * 4 + j;
-      acc[i][j] =
-          (d_state_out && r < dk && c < dv) ? d_state_out[((size_t)bh * dk + r) * dv + c] : 0.f;
+      acc[i][j] = (first && r < dk && c < dv) ? first[((size_t)bh * dk + r) * dv + c] : 0.f;
     }
-  for (int ci = nc - 1; ci >= 0; --ci) {
-    float* G = gws + ((size_t)bh * nc + ci) * dk * dv;
+  for (int t = 0; t < nc; ++t) {
+    const int ci = FWD ? t : nc - 1 - t;
+    float* S = slots + ((size_t)bh * nc + ci) * dk * dv;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int r = r0 + ty * 4 + i, c = c0 + tx * 4 + j;
-        if (r < dk && c < dv) G[(size_t)r * dv + c] = acc[i][j];
+        if (r < dk && c < dv) S[(size_t)r * dv + c] = acc[i][j];
       }
     const int s = ci * chunk;
     const int L = min(chunk, N - s);
@@ -74,36 +81,37 @@ grad_scan(const T* __restrict__ q, const T* __restrict__ dout, const float* __re
         const int jj = e / ST, x = e % ST;
         const int j = j0 + jj;
         const size_t tok = (size_t)bh * N + s + j;
-        float qv = 0.f, dvv = 0.f;
+        float av = 0.f, bv = 0.f;
         if (j < L) {
-          if (r0 + x < dk) qv = Elem<T>::ld(q + tok * dk + r0 + x);
-          if (c0 + x < dv) dvv = Elem<T>::ld(dout + tok * dv + c0 + x) * gpow(lg, j + 1);
+          if (r0 + x < dk) av = Elem<T>::ld(a + tok * dk + r0 + x);
+          if (c0 + x < dv)
+            bv = Elem<T>::ld(b + tok * dv + c0 + x) * gpow(lg, FWD ? L - 1 - j : j + 1);
         }
-        qs[jj][x] = qv;
-        ds[jj][x] = dvv;
+        as[jj][x] = av;
+        bs[jj][x] = bv;
       }
       __syncthreads();
 #pragma unroll 4
       for (int jj = 0; jj < SJ; ++jj) {
-        float a[4], b[4];
+        float av[4], bv[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) a[i] = qs[jj][ty * 4 + i];
+        for (int i = 0; i < 4; ++i) av[i] = as[jj][ty * 4 + i];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) b[j] = ds[jj][tx * 4 + j];
+        for (int j = 0; j < 4; ++j) bv[j] = bs[jj][tx * 4 + j];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
       }
     }
   }
-  if (d_state_in) {
+  if (last) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int r = r0 + ty * 4 + i, c = c0 + tx * 4 + j;
-        if (r < dk && c < dv) d_state_in[((size_t)bh * dk + r) * dv + c] = acc[i][j];
+        if (r < dk && c < dv) last[((size_t)bh * dk + r) * dv + c] = acc[i][j];
       }
   }
 }
@@ -274,7 +282,7 @@ template <typename T>
 cudaError_t backward_t(const void* q, const void* k, const void* v, const float* gammas, int chunk,
                        const float* state_in, const void* dout, const float* d_state_out,
                        void* dq, void* dk_, void* dv_, float* d_state_in, int B, int H, int N,
-                       int dk, int dv, int dtype, void* ws, cudaStream_t st) {
+                       int dk, int dv, void* ws, cudaStream_t st) {
   chunk = work_chunk(chunk);
   const int nc = cdiv(N, chunk);
   const size_t slots = (size_t)B * H * nc;
@@ -282,17 +290,17 @@ cudaError_t backward_t(const void* q, const void* k, const void* v, const float*
   float* gws = rws + slots * dk * dv;
   float* pws = gws + slots * dk * dv;
   float* sws = pws + slots * chunk * chunk;
-  cudaError_t e = launch_simt_states(k, v, gammas, chunk, state_in, nullptr, B, H, N, dk, dv,
-                                     dtype, rws, st);
-  if (e != cudaSuccess) return e;
   const T* Q = static_cast<const T*>(q);
   const T* K = static_cast<const T*>(k);
   const T* V = static_cast<const T*>(v);
   const T* dO = static_cast<const T*>(dout);
-  dim3 g1(cdiv(dv, ST), cdiv(dk, ST), B * H);
-  grad_scan<T><<<g1, 256, 0, st>>>(Q, dO, gammas, chunk, d_state_out, d_state_in, gws, H, N, dk,
-                                   dv);
-  if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
+  const dim3 g1(cdiv(dv, ST), cdiv(dk, ST), B * H);
+  state_scan<T, true><<<g1, 256, 0, st>>>(K, V, gammas, chunk, state_in, nullptr, rws, H, N, dk,
+                                          dv);
+  state_scan<T, false><<<g1, 256, 0, st>>>(Q, dO, gammas, chunk, d_state_out, d_state_in, gws, H,
+                                           N, dk, dv);
+  cudaError_t e = cudaPeekAtLastError();
+  if (e != cudaSuccess) return e;
   const int nt = cdiv(chunk, GM);
   const dim3 gs(nc, nt * (nt + 1) / 2, B * H);
   chunk_scores<T><<<gs, 256, 0, st>>>(dO, V, gammas, chunk, pws, H, N, dv);
@@ -324,9 +332,9 @@ cudaError_t launch_chunkwise_backward(const void* q, const void* k, const void* 
                                       cudaStream_t st) {
   if (dtype == RET_BF16)
     return bwd::backward_t<__nv_bfloat16>(q, k, v, gammas, chunk, state_in, dout, d_state_out, dq,
-                                          dk_, dv_, d_state_in, B, H, N, dk, dv, dtype, ws, st);
+                                          dk_, dv_, d_state_in, B, H, N, dk, dv, ws, st);
   return bwd::backward_t<float>(q, k, v, gammas, chunk, state_in, dout, d_state_out, dq, dk_, dv_,
-                                d_state_in, B, H, N, dk, dv, dtype, ws, st);
+                                d_state_in, B, H, N, dk, dv, ws, st);
 }
 
 }  // namespace ret
