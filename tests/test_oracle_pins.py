@@ -467,6 +467,19 @@ def test_rotation_invariants():
         oracle.rotate(np.zeros((2, 3)), np.zeros(1))
 
 
+def test_rotation_of_a_span_is_a_slice_of_the_whole():
+    """A span that starts at position s, rotated with pos0 = s, gives the
+    same rows as the whole sequence rotated from 0 (what a caller does when a
+    sequence is split across GPUs, or when decoding token s)."""
+    rng = np.random.default_rng(33)
+    x = rng.standard_normal((2, 3, 40, 12))
+    th = rng.uniform(0.0, 2.0, 6)
+    whole = oracle.rotate(x, th, 0)
+    for s0, s1 in ((0, 7), (7, 23), (23, 40), (39, 40)):
+        np.testing.assert_allclose(oracle.rotate(x[..., s0:s1, :], th, s0), whole[..., s0:s1, :],
+                                   rtol=0, atol=1e-13)
+
+
 def _rotate_mutant(x, theta, pos0, mutation):
     """A copy of the oracle's rotation with one planted mistake."""
     x = np.asarray(x, dtype=np.float64)
