@@ -17,6 +17,11 @@ spans.  Each rank
 Step 4 recomputes the chunk states of the span with the incoming state, so the
 states phase runs twice; the exchange is the only communication.
 
+With the xPos rotation (same page, core components, item 3: a complex
+rotation of Q and K by position), q and k of a span are rotated from the
+span's own start position before step 1, so the span lengths are gathered
+first; every rank then holds the rows the unsplit sequence would have.
+
 The steps are exposed separately (`local_end_state`, `span_output`) so that
 callers can run them across processes themselves; `chunkwise_sequence_parallel`
 runs all four with torch.distributed.  The arithmetic of every step is the
@@ -40,6 +45,10 @@ class CudaOps:
         s = torch.empty((B, H, dk, dv), dtype=torch.float32, device=k.device)
         chunkwise_states(k, v, gammas, chunk, ws, state_out=s)
         return s
+
+    def rotate(self, x, theta, pos0):
+        from . import rotate
+        return rotate(x, theta, pos0)
 
     def combine(self, locals_, spans, r, gammas, state0):
         from . import state_combine
@@ -70,25 +79,31 @@ def span_output(q, k, v, gammas, chunk, locals_, spans, rank, state0=None, gn_ep
 
 
 def chunkwise_sequence_parallel(q, k, v, gammas, chunk, group=None, state0=None, gn_eps=None,
-                                gate=None, return_state=False, ops=None):
+                                gate=None, return_state=False, ops=None, theta=None, pos0=0):
     """All four steps over the ranks of `group` (torch.distributed): q, k, v
     (and gate) are this rank's span, [B,H,N_rank,d]; every rank passes the
     same gammas, chunk, state0 (the state entering the whole sequence, or
-    None) and options.  Returns this span's o, and with return_state the end
-    state of the whole sequence (the same on every rank)."""
+    None) and options.  With theta ([d_k/2] angles) q and k are rotated
+    first, the first token of the whole sequence sitting at position pos0.
+    Returns this span's o, and with return_state the end state of the whole
+    sequence (the same on every rank)."""
     import torch
     import torch.distributed as dist
 
     ops = ops or CudaOps()
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
-    s_loc = ops.local_end_state(q, k, v, gammas, chunk).contiguous()
-    n = torch.tensor([q.shape[2]], dtype=torch.int64, device=s_loc.device)
+    n = torch.tensor([q.shape[2]], dtype=torch.int64, device=q.device)
     ns = [torch.empty_like(n) for _ in range(world)]
     dist.all_gather(ns, n, group=group)
+    spans = [int(x.item()) for x in ns]
+    if theta is not None:
+        start = pos0 + sum(spans[:rank])
+        q = ops.rotate(q, theta, start)
+        k = ops.rotate(k, theta, start)
+    s_loc = ops.local_end_state(q, k, v, gammas, chunk).contiguous()
     gathered = [torch.empty_like(s_loc) for _ in range(world)]
     dist.all_gather(gathered, s_loc, group=group)
-    spans = [int(x.item()) for x in ns]
     locals_ = torch.stack(gathered)
     return span_output(q, k, v, gammas, chunk, locals_, spans, rank, state0=state0,
                        gn_eps=gn_eps, gate=gate, return_state=return_state, ops=ops)

@@ -23,6 +23,9 @@ class OracleOps:
         _, s = oracle.chunkwise(q.numpy(), k.numpy(), v.numpy(), gammas.numpy(), chunk)
         return torch.from_numpy(s)
 
+    def rotate(self, x, theta, pos0):
+        return torch.from_numpy(oracle.rotate(x.numpy(), theta.numpy(), pos0))
+
     def combine(self, locals_, spans, r, gammas, state0):
         # the chunk recurrence at span granularity: S <- gamma^N S + S_local
         g = gammas.numpy()[None, :, None, None]
@@ -58,7 +61,7 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, out, rotated=False):
     import torch.distributed as dist
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
@@ -72,28 +75,42 @@ def _worker(rank, world, port, out):
             t(inp["q"].exact), t(inp["k"].exact), t(inp["v"].exact),
             torch.from_numpy(inp["gammas"].astype(np.float64)), 16,
             state0=torch.from_numpy(inp["state"].exact), gn_eps=1e-5, gate=t(gate),
-            return_state=True, ops=OracleOps())
+            return_state=True, ops=OracleOps(),
+            theta=torch.from_numpy(_theta()) if rotated else None, pos0=POS0)
         out[rank] = (a, b, o.numpy(), s.numpy())
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_spans_over_gloo_match_the_unsplit_sequence(world):
+POS0 = 1000
+
+
+def _theta():
+    return wl.rotation_angles(8, seed=4).astype(np.float64)
+
+
+@pytest.mark.parametrize("world,rotated", [(2, False), (3, False), (2, True), (3, True)])
+def test_spans_over_gloo_match_the_unsplit_sequence(world, rotated):
+    """With rotated, q and k of each span are rotated from the span's start
+    position (POS0 + the tokens before it) and must match the unsplit
+    sequence rotated from POS0."""
     assert sum(SPANS[world]) == 150
     ctx = mp.get_context("spawn")
     mgr = ctx.Manager()
     out = mgr.dict()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, out, rotated))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
         p.join(120)
         assert p.exitcode == 0
     inp, gate = _inputs()
-    o_ref, s_ref = oracle.chunkwise(inp["q"].exact, inp["k"].exact, inp["v"].exact,
-                                    inp["gammas"], 16, inp["state"].exact)
+    q, k = inp["q"].exact, inp["k"].exact
+    if rotated:
+        q, k = oracle.rotate(q, _theta(), POS0), oracle.rotate(k, _theta(), POS0)
+    o_ref, s_ref = oracle.chunkwise(q, k, inp["v"].exact, inp["gammas"], 16, inp["state"].exact)
     o_ref = oracle.gated(oracle.group_norm(o_ref, 1e-5), gate)
     for r in range(world):
         a, b, o, s = out[r]
