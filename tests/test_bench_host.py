@@ -33,6 +33,17 @@ def test_ragged_chunks_count_exact_lengths():
     assert F == (512 * 513 + 488 * 489) * 5 + 2 * (2 * 2 * 3 * 1000)
 
 
+def test_phase_split_and_single_chunk_agree_with_the_whole():
+    """The two phases' flops add up to the whole call, and one chunk covering
+    the sequence (no state in or out) is the parallel form's causal count."""
+    for args in ((8, 16, 8192, 256, 512, 512, False, False), (1, 2, 1000, 64, 96, 128, True, True),
+                 (2, 3, 77, 8, 16, 37, True, False)):
+        st, out = bench.chunkwise_phase_flops(*args)
+        assert st + out == bench.chunkwise_flops(*args)
+    assert bench.chunkwise_flops(8, 8, 2048, 256, 256, 2048) == \
+        bench.parallel_flops(8, 8, 2048, 256, 256)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
