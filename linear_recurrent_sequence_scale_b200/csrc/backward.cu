@@ -228,15 +228,16 @@ chunk_grads(const T* __restrict__ b1, const T* __restrict__ a2, const float* __r
   const float* P = scores + ((size_t)bh * gridDim.x + ci) * chunk * chunk;
   const T* B1 = b1 + ((size_t)bh * N + cs) * ncol;
   float acc[4][4] = {};
+  auto lb1 = [&](int k, int c) {
+    return c0 + c < ncol ? Elem<T>::ld(B1 + (size_t)k * ncol + c0 + c) : 0.f;
+  };
   if (MODE == 0)
     tile_product<true, false>(
-        t, [&](int r, int k) { return r0 + r < L ? P[(size_t)(r0 + r) * chunk + k] : 0.f; },
-        [&](int k, int c) { return c0 + c < ncol ? Elem<T>::ld(B1 + (size_t)k * ncol + c0 + c) : 0.f; },
+        t, [&](int r, int k) { return r0 + r < L ? P[(size_t)(r0 + r) * chunk + k] : 0.f; }, lb1,
         0, min(L, r0 + GM), acc);
   else
     tile_product<false, false>(
-        t, [&](int r, int k) { return r0 + r < L ? P[(size_t)k * chunk + r0 + r] : 0.f; },
-        [&](int k, int c) { return c0 + c < ncol ? Elem<T>::ld(B1 + (size_t)k * ncol + c0 + c) : 0.f; },
+        t, [&](int r, int k) { return r0 + r < L ? P[(size_t)k * chunk + r0 + r] : 0.f; }, lb1,
         r0, L, acc);
   if (MODE != 0 || ci > 0 || has_r0) {
     const float lg = log2f(gammas[bh % H]);
@@ -307,9 +308,9 @@ cudaError_t backward_t(const void* q, const void* k, const void* v, const float*
   chunk_scores<T><<<gs, 256, 0, st>>>(Q, K, gammas, chunk, sws, H, N, dk);
   if ((e = cudaPeekAtLastError()) != cudaSuccess) return e;
   const dim3 gk(nc, nt * cdiv(dk, GN_), B * H), gv(nc, nt * cdiv(dv, GN_), B * H);
-  const int r0 = state_in != nullptr;
-  chunk_grads<T, 0><<<gk, 256, 0, st>>>(K, dO, pws, rws, r0, gammas, chunk, static_cast<T*>(dq),
-                                        H, N, dv, dk, dk, dv);
+  const int has_r0 = state_in != nullptr;
+  chunk_grads<T, 0><<<gk, 256, 0, st>>>(K, dO, pws, rws, has_r0, gammas, chunk,
+                                        static_cast<T*>(dq), H, N, dv, dk, dk, dv);
   chunk_grads<T, 1><<<gk, 256, 0, st>>>(Q, V, pws, gws, 1, gammas, chunk, static_cast<T*>(dk_), H,
                                         N, dv, dk, dk, dv);
   chunk_grads<T, 2><<<gv, 256, 0, st>>>(dO, K, sws, gws, 1, gammas, chunk, static_cast<T*>(dv_), H,
