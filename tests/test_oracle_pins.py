@@ -94,6 +94,17 @@ def test_hand_worked_group_norm():
     np.testing.assert_allclose(out, g["out"], rtol=0, atol=1e-15)
 
 
+def test_hand_worked_backward():
+    g = _golden()["backward"]
+    one = lambda x: np.asarray(x, dtype=np.float64).reshape(1, 1, 1, 1)
+    dq, dk, dv, ds = oracle.backward(_seq(g["q"]), _seq(g["k"]), _seq(g["v"]), [g["gamma"]],
+                                     _seq(g["d_o"]), one(g["state_in"]), one(g["d_state_out"]))
+    np.testing.assert_allclose(dq[0, 0, :, 0], g["dq"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(dk[0, 0, :, 0], g["dk"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(dv[0, 0, :, 0], g["dv"], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(ds[0, 0, 0, 0], g["d_state_in"], rtol=0, atol=1e-14)
+
+
 # --- P2: decay mask against brute force --------------------------------------
 
 @pytest.mark.parametrize("gamma", [0.0, 0.3, 0.5, 0.96875, 1.0 - 2.0 ** -20, 1.0])
