@@ -523,3 +523,40 @@ def _rotate_mutant(x, theta, pos0, mutation):
                                       "half_split_pairs", "rows_not_positions"])
 def test_rotation_pins_catch_planted_mistakes(mutation):
     assert not _rotation_pins_hold(lambda x, t, p: _rotate_mutant(x, t, p, mutation))
+
+
+def _backward_mutant(q, k, v, gam, d_o, s_in, d_s, mutation):
+    """A copy of the oracle's backward for one (b, h) with one planted mistake."""
+    Q, K, V, dO = q[0, 0], k[0, 0], v[0, 0], d_o[0, 0]
+    S, dS = s_in[0, 0], d_s[0, 0]
+    N = Q.shape[0]
+    n = np.arange(N)
+    g = float(gam[0])
+    D = oracle.decay_mask(g, N)
+    xi = g ** (n + 1.0)
+    z = g ** (N - 1.0 - n)
+    if mutation == "xi_exponent":
+        xi = g ** n
+    if mutation == "zeta_exponent":
+        z = g ** (N - n)
+    A = (Q @ K.T) * D
+    dA = (dO @ V.T) * (np.ones_like(D) if mutation == "mask_dropped" else D)
+    dq = dA @ K + xi[:, None] * (dO @ S.T)
+    dk = dA.T @ Q + z[:, None] * (V @ dS.T)
+    dv = (A if mutation == "untransposed_a" else A.T) @ dO + z[:, None] * (K @ dS)
+    ds = (Q * xi[:, None]).T @ dO + (0.0 if mutation == "no_state_carry" else g ** N * dS)
+    return dq, dk, dv, ds
+
+
+@pytest.mark.parametrize("mutation", ["xi_exponent", "zeta_exponent", "mask_dropped",
+                                      "untransposed_a", "no_state_carry"])
+def test_backward_pins_catch_planted_mistakes(mutation):
+    g = _golden()["backward"]
+    one = lambda x: np.asarray(x, dtype=np.float64).reshape(1, 1, 1, 1)
+    got = _backward_mutant(_seq(g["q"]), _seq(g["k"]), _seq(g["v"]), [g["gamma"]],
+                           _seq(g["d_o"]), one(g["state_in"]), one(g["d_state_out"]), mutation)
+    want = (g["dq"], g["dk"], g["dv"], [g["d_state_in"]])
+    clean = _backward_mutant(_seq(g["q"]), _seq(g["k"]), _seq(g["v"]), [g["gamma"]],
+                             _seq(g["d_o"]), one(g["state_in"]), one(g["d_state_out"]), None)
+    assert all(np.allclose(np.ravel(a), b, rtol=0, atol=1e-12) for a, b in zip(clean, want))
+    assert any(not np.allclose(np.ravel(a), b, rtol=0, atol=1e-9) for a, b in zip(got, want))
