@@ -560,3 +560,89 @@ def test_backward_pins_catch_planted_mistakes(mutation):
                              _seq(g["d_o"]), one(g["state_in"]), one(g["d_state_out"]), None)
     assert all(np.allclose(np.ravel(a), b, rtol=0, atol=1e-12) for a, b in zip(clean, want))
     assert any(not np.allclose(np.ravel(a), b, rtol=0, atol=1e-9) for a, b in zip(got, want))
+
+
+# --- the parity checker ------------------------------------------------------
+# Every parity assertion divides ||x - ref||_F by ||ref||_F.  The values below
+# are worked by hand, and each planted mistake in a copy of the quotient
+# (a difference of norms, no square root, the wrong denominator, zero for a
+# zero reference, a max-norm) fails at least one of them.
+
+REL_FROBENIUS_CASES = [
+    # x, ref, value worked by hand
+    ([0.0, 0.0], [3.0, 4.0], 1.0),                    # ||(-3,-4)|| / ||(3,4)|| = 5/5
+    ([1.0, 1.0], [1.0, 2.0], 1.0 / np.sqrt(5.0)),     # ||(0,-1)|| / sqrt(1 + 4)
+    ([1.0, 2.0], [1.0, 1.0], 1.0 / np.sqrt(2.0)),     # divided by the reference, not by x
+    ([[1.0, 0.0], [0.0, 1.0]], [[2.0, 0.0], [0.0, 2.0]], 0.5),   # sqrt(2) / sqrt(8)
+    ([-3.0, -4.0], [3.0, 4.0], 2.0),                  # ||(-6,-8)|| / 5: the sign counts
+    ([3.0, 4.0], [3.0, 4.0], 0.0),
+    ([0.0, 0.0], [0.0, 0.0], 0.0),                    # both zero
+    ([0.5, 0.0], [0.0, 0.0], np.inf),                 # any error against a zero reference
+]
+
+
+def _rel_frobenius_pins_hold(fn):
+    for x, ref, want in REL_FROBENIUS_CASES:
+        got = fn(np.asarray(x), np.asarray(ref))
+        if np.isinf(want):
+            if not np.isinf(got):
+                return False
+        elif not np.isclose(got, want, rtol=1e-14, atol=0.0):
+            return False
+    return True
+
+
+def _rel_frobenius_mutant(x, ref, mutation):
+    x, ref = np.asarray(x, np.float64), np.asarray(ref, np.float64)
+    num = np.linalg.norm((x - ref).ravel())
+    den = np.linalg.norm(ref.ravel())
+    if mutation == "difference_of_norms":
+        num = abs(np.linalg.norm(x.ravel()) - den)
+    if mutation == "no_square_root":
+        num, den = num ** 2, den ** 2
+    if mutation == "divided_by_x":
+        den = np.linalg.norm(x.ravel())
+    if mutation == "max_norm":
+        num, den = np.abs(x - ref).max(), np.abs(ref).max()
+    if den == 0.0:
+        if mutation == "zero_reference_passes":
+            return 0.0
+        return 0.0 if num == 0.0 else float("inf")
+    return float(num / den)
+
+
+def test_rel_frobenius_hand_worked():
+    assert _rel_frobenius_pins_hold(oracle.rel_frobenius)
+
+
+@pytest.mark.parametrize("mutation", ["difference_of_norms", "no_square_root", "divided_by_x",
+                                      "max_norm", "zero_reference_passes"])
+def test_rel_frobenius_pins_catch_planted_mistakes(mutation):
+    assert _rel_frobenius_pins_hold(lambda x, r: _rel_frobenius_mutant(x, r, None))
+    assert not _rel_frobenius_pins_hold(lambda x, r: _rel_frobenius_mutant(x, r, mutation))
+
+
+def test_parity_blocks_find_a_local_error():
+    """A defect confined to one 128-row tile of one head, diluted below the
+    tolerance in the whole-output figure, is reported at full size by the
+    per-tile check the GPU tests use."""
+    from parity_check import worst, worst_rel
+    rng = np.random.default_rng(5)
+    ref = rng.standard_normal((2, 3, 8192, 64))
+    x = ref.copy()
+    x[1, 2, 1024:1152] *= 1.15                  # one tile 15% off
+    assert oracle.rel_frobenius(x, ref) < 2e-2  # lost in the whole
+    where, e = worst(x, ref)
+    assert where == "(b,h)=(1, 2) rows 1024:1152" and np.isclose(e, 0.15, rtol=1e-12)
+    assert worst_rel(ref, ref) == 0.0
+    # a head that is wrong as a whole, and a decode row ([B,H,d] layout)
+    y = ref.copy()
+    y[0, 1] *= 1.01
+    assert np.isclose(worst_rel(y, ref), 0.01, rtol=1e-12)
+    d = rng.standard_normal((4, 16, 512))
+    dd = d.copy()
+    dd[3, 9] = 0.0
+    assert worst(dd, d)[0] == "(b,h)=(3, 9)" and worst_rel(dd, d) == 1.0
+    nan = ref.copy()
+    nan[0, 0, 5, 5] = np.nan
+    assert worst_rel(nan, ref) == np.inf
