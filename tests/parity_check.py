@@ -79,8 +79,21 @@ def worst(x, ref, tile=TILE):
     return max(blocks(x, ref, tile), key=lambda b: (np.isnan(b[1]), b[1]))
 
 
+class WorstError(float):
+    """A rel-Frobenius error that also says where it was found (shown when an
+    assertion on it fails)."""
+
+    def __new__(cls, value, where):
+        obj = super().__new__(cls, value)
+        obj.where = where
+        return obj
+
+    def __repr__(self):
+        return f"{float(self):.4g} (worst at {self.where})"
+
+
 def worst_rel(x, ref, tile=TILE) -> float:
     """The largest rel-Frobenius error over the whole array, each (batch,
     head) and each `tile`-row block (NaN counts as the worst)."""
-    e = worst(x, ref, tile)[1]
-    return float("inf") if np.isnan(e) else e
+    where, e = worst(x, ref, tile)
+    return WorstError(float("inf") if np.isnan(e) else e, where)

@@ -6,6 +6,7 @@ import pytest
 
 import oracle
 from linear_recurrent_sequence_scale_b200 import workloads as wl
+from parity_check import worst_rel
 
 pytestmark = pytest.mark.gpu
 
@@ -30,5 +31,5 @@ def test_bounded_wait_runs_out_and_reports():
     o = ret.chunkwise(q, k, v, g, 128)
     torch.cuda.synchronize()
     o_ref, _ = oracle.chunkwise(inp["q"].exact, inp["k"].exact, inp["v"].exact, inp["gammas"], 128)
-    assert oracle.rel_frobenius(wl.from_torch(o), o_ref) <= 2e-2
+    assert worst_rel(wl.from_torch(o), o_ref) <= 2e-2
     assert ret.device_error() == 0

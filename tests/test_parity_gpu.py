@@ -1,8 +1,10 @@
 """CUDA path against the CPU oracle, element by element on the same inputs.
 
-Tolerances (rel-Frobenius over the whole output): 1e-5 for float32 inputs,
-2e-2 for bf16 inputs with float32 accumulation, 1e-4 for every float32 state
-returned.  bf16 inputs are rounded once by the input generator and the oracle
+Tolerances (rel-Frobenius): 1e-5 for float32 inputs, 2e-2 for bf16 inputs
+with float32 accumulation, 1e-4 for every float32 state returned.  Each holds
+for the whole output and also for every (batch, head) slice and every
+128-row tile of it, so that an error confined to one tile, ring slot or chunk
+boundary is not diluted by the rest of the output.  bf16 inputs are rounded once by the input generator and the oracle
 consumes exactly those rounded values in float64.
 """
 import numpy as np
@@ -10,6 +12,7 @@ import pytest
 
 import oracle
 from linear_recurrent_sequence_scale_b200 import workloads as wl
+from parity_check import worst_rel
 
 pytestmark = pytest.mark.gpu
 
@@ -48,7 +51,9 @@ def _gam(torch, g):
 
 
 def _rel(x, ref):
-    return oracle.rel_frobenius(wl.from_torch(x) if not isinstance(x, np.ndarray) else x, ref)
+    """The worst rel-Frobenius error over the whole output, each (batch, head)
+    and each 128-row tile (see parity_check)."""
+    return worst_rel(wl.from_torch(x) if not isinstance(x, np.ndarray) else x, ref)
 
 
 def _ref_chunkwise(inp, chunk, gn, with_state_in):
@@ -132,6 +137,27 @@ def test_chunkwise_without_state_out_and_in_place(torch_cuda, ret):
     assert _rel(s, s_ref) <= STATE_TOL
 
 
+@pytest.mark.parametrize("N", [1, 200, 512])
+def test_single_chunk_state_out_read_right_after_the_call(torch_cuda, ret, N):
+    """One chunk and no incoming state: no output tile reads a chunk state,
+    so nothing inside the output kernel waits for the state scan.  The call
+    must still complete only after the scan: the final state is consumed by
+    the next operation on the same stream, with no synchronisation between."""
+    torch = torch_cuda
+    B, H, dk, dv, C = 2, 3, 256, 512, 512
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=900 + N)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    o_ref, s_ref = _ref_chunkwise(inp, C, 1e-5, False)
+    for _ in range(3):
+        s = torch.full((B, H, dk, dv), float("nan"), dtype=torch.float32, device="cuda")
+        o, _ = ret.chunkwise(q, k, v, g, C, state_out=s, gn_eps=1e-5)
+        s_next = s * 1.0   # the next stream operation reads the state at once
+        torch.cuda.synchronize()
+        assert _rel(o, o_ref) <= TOL["bf16"]
+        assert _rel(s_next, s_ref) <= STATE_TOL
+
+
 @pytest.mark.parametrize("dt,chunk,gn", [("bf16", 256, 1e-5), ("f32", 100, None)])
 def test_chunkwise_in_two_phases(torch_cuda, ret, dt, chunk, gn):
     """ret_chunkwise_states then ret_chunkwise_output: the oracle's result, and
@@ -157,9 +183,11 @@ def test_chunkwise_in_two_phases(torch_cuda, ret, dt, chunk, gn):
 
 @pytest.mark.parametrize("gn", [None, 1e-5])
 def test_chunkwise_strong_and_weak_decays(torch_cuda, ret, gn):
-    """Decays on both sides of gamma^chunk = 2^-64: the kernel folds xi into
-    the mask and the epilogue for the weak ones and rescales Q for the strong
-    ones (0.5^256 and 0); both must match the oracle, with a state entering."""
+    """Weak and strong decays with a state entering: gamma^256 runs from
+    0.77 (0.999) down to 0.5^256 (below float32's range, so xi and the mask
+    flush to zero) and 0 (where 0^0 = 1 keeps the diagonal).  The kernel
+    scales each Q row by xi in place for every decay; all must match the
+    oracle."""
     torch = torch_cuda
     B, H, N, dk, dv, C = 1, 4, 700, 128, 256, 256
     gam = [0.5, 0.9, 0.999, 0.0]
@@ -173,28 +201,57 @@ def test_chunkwise_strong_and_weak_decays(torch_cuda, ret, gn):
     assert _rel(s, s_ref) <= STATE_TOL
 
 
+def _offset_v(inp, dv, offset):
+    """v with every fourth 32-column group spread 30x and a common offset:
+    the retention output rows then carry a mean far from zero."""
+    col = np.where((np.arange(dv) // 32) % 4 == 0, 30.0, 1.0)
+    return wl.from_values(inp["v"].exact * col + offset, "bf16")
+
+
 def test_groupnorm_far_from_zero_mean(torch_cuda, ret):
-    """GroupNorm where every output row carries a large common offset and the
-    32-column groups differ in spread by 30x: the normalised deviations must
-    still come out to bf16 accuracy (chunkwise with two d_v slices, and the
-    parallel form with one)."""
+    """GroupNorm where every output row carries a large common offset (row
+    means about 20x the spread) and the 32-column groups differ in spread by
+    30x: the normalised deviations must still come out to bf16 accuracy in
+    every tile (parallel form, one 256-column slice)."""
+    torch = torch_cuda
+    B, H, N, dk, dv = 1, 2, 600, 128, 256
+    inp = wl.make_inputs(B, H, N, dk, 512, "bf16", seed=41)
+    v = _offset_v(inp, 512, 40.0)
+    q, k, vd = _dev(inp["q"]), _dev(inp["k"]), _dev(v)
+    g = _gam(torch, inp["gammas"])
+    vs = vd[..., :dv].contiguous()
+    op = ret.parallel(q, k, vs, g, gn_eps=1e-5)
+    p_ref, _ = oracle.parallel(inp["q"].exact, inp["k"].exact, v.exact[..., :dv], inp["gammas"])
+    p_ref = oracle.group_norm(p_ref, 1e-5)
+    torch.cuda.synchronize()
+    assert _rel(op, p_ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("offset", [8.0, 40.0])
+def test_chunkwise_groupnorm_far_from_zero_mean(torch_cuda, ret, offset):
+    """The same stress for the chunkwise form (two d_v slices, three chunks).
+    Its cross-chunk term reads the chunk state as bf16, and that rounding
+    (relative 2^-9 of every state element) is not removed by the GroupNorm's
+    mean subtraction: after normalisation its error grows with the ratio of
+    the row means to the row spread, about 1.4e-3 per unit of that ratio
+    (float64 emulation of the rounding).  At offset 8 (ratio 4) every tile
+    meets the bf16 tolerance; at offset 40 (ratio 20) the whole output does,
+    and every tile stays within the bound that ratio gives (5e-2)."""
     torch = torch_cuda
     B, H, N, dk, dv, C = 1, 2, 600, 128, 512, 256
     inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=41)
-    col = np.where((np.arange(dv) // 32) % 4 == 0, 30.0, 1.0)
-    v = wl.from_values(inp["v"].exact * col + 40.0, "bf16")
+    v = _offset_v(inp, dv, offset)
     q, k, vd = _dev(inp["q"]), _dev(inp["k"]), _dev(v)
     g = _gam(torch, inp["gammas"])
     o = ret.chunkwise(q, k, vd, g, C, gn_eps=1e-5)
     o_ref, _ = oracle.chunkwise(inp["q"].exact, inp["k"].exact, v.exact, inp["gammas"], C)
     o_ref = oracle.group_norm(o_ref, 1e-5)
-    vs = vd[..., :256].contiguous()
-    op = ret.parallel(q, k, vs, g, gn_eps=1e-5)
-    p_ref, _ = oracle.parallel(inp["q"].exact, inp["k"].exact, v.exact[..., :256], inp["gammas"])
-    p_ref = oracle.group_norm(p_ref, 1e-5)
     torch.cuda.synchronize()
-    assert _rel(o, o_ref) <= TOL["bf16"]
-    assert _rel(op, p_ref) <= TOL["bf16"]
+    if offset <= 8.0:
+        assert _rel(o, o_ref) <= TOL["bf16"]
+    else:
+        assert oracle.rel_frobenius(wl.from_torch(o), o_ref) <= TOL["bf16"]
+        assert _rel(o, o_ref) <= 5e-2
 
 
 # --- gated output: swish(G) (.) Y -----------------------------------------------
@@ -579,6 +636,45 @@ def test_rotate_decode_row_and_empty(torch_cuda, ret):
     _rotation_close(y, ref, x.exact, "bf16")
     e = torch.full((1, 2, 0, 64), 3.0, device="cuda")
     assert ret.rotate(e, torch.from_numpy(wl.rotation_angles(64)).cuda()).shape == e.shape
+
+
+@pytest.mark.parametrize("dt,gn,gated", [("bf16", None, False), ("bf16", 1e-5, True),
+                                         ("f32", None, False), ("f32", 1e-5, False)])
+def test_step_rotated_matches_rotation_then_step(torch_cuda, ret, dt, gn, gated):
+    """The decode step with the xPos rotation fused into its loads
+    (ret_step_rotated) at positions 0, 1, 4095 and 1.2e8, against the oracle's
+    rotation of q and k at that position followed by its recurrent step (and
+    GroupNorm and the gate where asked)."""
+    torch = torch_cuda
+    B, H, dk, dv = 2, 3, 256, 512
+    inp = wl.make_inputs(B, H, 1, dk, dv, dt, seed=61, with_state=True)
+    q, k, v = (_dev(inp[n])[:, :, 0].contiguous() for n in ("q", "k", "v"))
+    qe, ke, ve = (inp[n].exact[:, :, 0] for n in ("q", "k", "v"))
+    g = _gam(torch, inp["gammas"])
+    th = wl.rotation_angles(dk, seed=7)
+    tht = torch.from_numpy(th).cuda()
+    gate = wl.draw(np.random.Generator(np.random.PCG64(62)), (B, H, dv), 1.0, dt) if gated \
+        else None
+    for pos in (0, 1, 4095, 123456789):
+        state = _dev(inp["state"]).clone()
+        o = ret.step(q, k, v, g, state, gn_eps=gn, theta=tht, pos=pos,
+                     gate=None if gate is None else _dev(gate))
+        torch.cuda.synchronize()
+        qr = oracle.rotate(qe[:, :, None, :], th.astype(np.float64), pos)[:, :, 0]
+        kr = oracle.rotate(ke[:, :, None, :], th.astype(np.float64), pos)[:, :, 0]
+        o_ref, s_ref = oracle.step(qr, kr, ve, inp["gammas"], inp["state"].exact)
+        if gn is not None:
+            o_ref = oracle.group_norm(o_ref, gn)
+        if gate is not None:
+            o_ref = oracle.gated(o_ref, gate.exact)
+        assert _rel(o, o_ref) <= TOL[dt], pos
+        assert _rel(state, s_ref) <= STATE_TOL, pos
+    # without theta the call is the plain step
+    s1, s2 = _dev(inp["state"]).clone(), _dev(inp["state"]).clone()
+    o1 = ret.step(q, k, v, g, s1, gn_eps=gn)
+    o2 = ret.step(q, k, v, g, s2, gn_eps=gn, theta=None, pos=77)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
 
 
 def test_rotated_retention_matches_oracle(torch_cuda, ret):
