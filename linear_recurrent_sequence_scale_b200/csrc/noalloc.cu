@@ -9,11 +9,13 @@
 // instead of from the caller.
 //
 // The array lives in device memory of every GPU that loads the library, for
-// as long as the process runs.  Its device address is looked up once per
-// device, on the first call made with that device current.  All calls share
-// the one array, so calls that overlap on the GPU (different streams, or
-// different host threads on the same device) race on it and must be
-// serialised by the caller.  The array keeps whatever the last call left in
+// as long as the process runs.  Its device address is looked up on the first
+// call made with that device current, and kept once the lookup succeeds (a
+// failed lookup, say inside a stream capture, is retried on the next call).
+// The stream passed in must belong to the current device: the array used is
+// the current device's copy.  All calls share the one array, so calls that
+// overlap on the GPU (different streams, or different host threads on the
+// same device) race on it and must be serialised by the caller.  The array keeps whatever the last call left in
 // it; nothing needs to start at zero, because the chunkwise kernels write
 // every state slot before they read it.
 #include <cuda_runtime.h>
@@ -27,9 +29,21 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[RET_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
+// Per device: the array's device address once a lookup has succeeded (null
+// until then).  A failed lookup is not remembered, so a later call retries it.
 void* g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
-std::once_flag g_scratch_once[kMaxDevices];
+std::mutex g_scratch_mu[kMaxDevices];
+
+// This device's copy of the array (the current device), or null if the
+// runtime could not give its address.
+void* scratch_for(int dev) {
+  std::lock_guard<std::mutex> lock(g_scratch_mu[dev]);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess) g_scratch_ptr[dev] = p;
+  }
+  return g_scratch_ptr[dev];
+}
 
 }  // namespace
 
@@ -44,11 +58,9 @@ extern "C" int ret_chunkwise_noalloc(const void* q, const void* k, const void* v
   if (cudaGetDevice(&dev) != cudaSuccess) return RET_ECUDA;
   if (dev < 0 || dev >= kMaxDevices) return RET_EUNSUPPORTED;
   // Host code may not use the array's name as an address: ask the runtime
-  // for this device's copy (once per device, with the device current).
-  std::call_once(g_scratch_once[dev], [dev]() {
-    g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_ptr[dev], g_noalloc_scratch);
-  });
-  if (g_scratch_err[dev] != cudaSuccess) return RET_ECUDA;
+  // for this device's copy (with the device current; cached once found).
+  void* scratch = scratch_for(dev);
+  if (!scratch) return RET_ECUDA;
   return ret_chunkwise(q, k, v, gammas, chunk, state_in, state_out, o, B, H, N, dk, dv, dtype,
-                       gn_eps, g_scratch_ptr[dev], RET_NOALLOC_SCRATCH_BYTES, stream);
+                       gn_eps, scratch, RET_NOALLOC_SCRATCH_BYTES, stream);
 }

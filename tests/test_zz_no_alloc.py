@@ -3,7 +3,8 @@ allocate device memory (a plugin whose host runtime owns all device memory,
 or a loop that must not call cudaMalloc).  It takes its scratch from a fixed
 array inside the library, so its results must equal those of ret_chunkwise
 given a caller-allocated workspace, call after call, whatever the previous
-call left in the shared array.
+call left in the shared array, and match the CPU oracle on their own (so a
+fault shared by the two entry points does not pass unseen).
 
 This file is collected last on purpose: a run that stops at the first
 failure has run every other test before it.
@@ -15,6 +16,7 @@ import pytest
 
 import oracle
 from linear_recurrent_sequence_scale_b200 import workloads as wl
+from parity_check import worst_rel
 
 pytestmark = pytest.mark.gpu
 
@@ -53,8 +55,15 @@ def test_noalloc_matches_the_workspace_entry_point_on_consecutive_calls():
                                        B, H, N, dk, dv, code, -1.0 if gn is None else gn, stream)
         assert st == ret.RET_OK, ret.status_string(st)
         torch.cuda.synchronize()
-        assert oracle.rel_frobenius(wl.from_torch(o), wl.from_torch(o_ref)) <= TOL[dt]
-        assert oracle.rel_frobenius(wl.from_torch(s), wl.from_torch(s_ref)) <= STATE_TOL
+        assert worst_rel(wl.from_torch(o), wl.from_torch(o_ref)) <= TOL[dt]
+        assert worst_rel(wl.from_torch(s), wl.from_torch(s_ref)) <= STATE_TOL
+        # and against the oracle directly
+        o_or, s_or = oracle.chunkwise(inp["q"].exact, inp["k"].exact, inp["v"].exact,
+                                      inp["gammas"], C, inp["state"].exact if with_s0 else None)
+        if gn is not None:
+            o_or = oracle.group_norm(o_or, gn)
+        assert worst_rel(wl.from_torch(o), o_or) <= TOL[dt]
+        assert worst_rel(wl.from_torch(s), s_or) <= STATE_TOL
         assert ret.device_error() == 0
 
 
