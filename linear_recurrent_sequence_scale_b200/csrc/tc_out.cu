@@ -715,6 +715,12 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  // Launched after the state scan, this grid may start before the scan ends.
+  // Every CTA waits for it before leaving, so the call completes only after
+  // the scan has written everything, the final state included, even when no
+  // tile read a chunk state (one chunk, no incoming state).  Without a
+  // programmatic dependency the wait returns at once.
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
   if (p.nslices > 1) cluster_sync_all();  // no CTA leaves while its peer may touch its smem
 }
 
