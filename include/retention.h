@@ -151,6 +151,9 @@ RET_API int ret_chunkwise_output(const void* q, const void* k, const void* v, co
  *     rejected with RET_EWORKSPACE before anything runs.
  *   - The first call on each device looks the array's device address up (with
  *     that device current); make that first call before any stream capture.
+ *     A failed lookup returns RET_ECUDA and is retried by the next call.
+ *   - `stream` must belong to the current device, whose copy of the array
+ *     the call uses.
  *   - Every call shares the one array: calls that overlap on the GPU race on
  *     it and must be serialised by the caller.  Nothing in it needs to start
  *     at zero; it keeps the last call's contents.
@@ -203,6 +206,26 @@ RET_API int ret_chunkwise_output_gated(const void* q, const void* k, const void*
 RET_API int ret_step_gated(const void* q, const void* k, const void* v, const float* gammas,
                    float* state, const void* gate, void* o, int B, int H, int dk, int dv,
                    int dtype, float gn_eps, void* stream);
+
+/*
+ * One recurrent decode step with the xPos rotation of q and k fused into it
+ * ("RetNet - Retentive Network - A Successor to Transformer for LLMs", core
+ * components, item 3: xPos puts relative position into Q and K as a complex
+ * rotation).  The token sits at sequence position `pos`; as q and k are read,
+ * channel pair c, (x[2c], x[2c+1]) as the real and imaginary parts of z_c,
+ * is multiplied by e^{i pos theta[c]} (the reading ret_rotate documents), so
+ * the step equals ret_rotate of q and k at pos0 = pos followed by
+ * ret_step_gated, without rounding the rotated q and k to the storage type
+ * and without writing them.
+ *   theta : device [dk/2] float32 angles (radians per position), or NULL
+ *           for no rotation (then exactly ret_step_gated).
+ *   pos   : 0 .. 2^53 (used only when theta is given).
+ * Other arguments, layouts and errors as for ret_step_gated.
+ */
+RET_API int ret_step_rotated(const void* q, const void* k, const void* v, const float* gammas,
+                     const float* theta, long long pos, float* state, const void* gate,
+                     void* o, int B, int H, int dk, int dv, int dtype, float gn_eps,
+                     void* stream);
 
 /*
  * State entering span r of a sequence split into spans held by different GPUs

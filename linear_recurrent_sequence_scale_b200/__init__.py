@@ -38,6 +38,8 @@ SIGNATURES = {
     "ret_chunkwise_output_gated": (_I, [_P, _P, _P, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _I,
                                         _F, _P, _S, _P]),
     "ret_step_gated": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P]),
+    "ret_step_rotated": (_I, [_P, _P, _P, _P, _P, ctypes.c_longlong, _P, _P, _P, _I, _I, _I, _I,
+                              _I, _F, _P]),
     "ret_state_combine": (_I, [_P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _P]),
     "ret_chunkwise_backward_workspace": (_S, [_I, _I, _I, _I, _I, _I, _I]),
     "ret_chunkwise_backward": (_I, [_P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I,
@@ -361,9 +363,10 @@ def rotate(x, theta, pos0=0, out=None):
     return out
 
 
-def step(q, k, v, gammas, state, gn_eps=None, out=None, gate=None):
-    """One recurrent decode step (ret_step; ret_step_gated with a gate [B,H,dv]):
-    state is updated in place; returns o.
+def step(q, k, v, gammas, state, gn_eps=None, out=None, gate=None, theta=None, pos=0):
+    """One recurrent decode step (ret_step; ret_step_gated with a gate [B,H,dv];
+    ret_step_rotated with theta [dk/2], q and k then rotated by pos * theta as
+    they are read): state is updated in place; returns o.
     q, k [B,H,dk]; v [B,H,dv]; state [B,H,dk,dv] float32."""
     torch = _torch()
     if q.dim() != 3:
@@ -382,7 +385,12 @@ def step(q, k, v, gammas, state, gn_eps=None, out=None, gate=None):
     gate = _gate(gate, q, (B, H, dv), dev)
     eps = -1.0 if gn_eps is None else float(gn_eps)
     lib = load_library()
-    if gate is None:
+    if theta is not None:
+        _check(theta, "theta", dtype=torch.float32, shape=(dk // 2,), device=dev)
+        s = lib.ret_step_rotated(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), _ptr(theta), int(pos),
+                                 _ptr(state), _ptr(gate), _ptr(out), B, H, dk, dv,
+                                 _dtype_code(q), eps, _stream(dev))
+    elif gate is None:
         s = lib.ret_step(_ptr(q), _ptr(k), _ptr(v), _ptr(gammas), _ptr(state), _ptr(out),
                          B, H, dk, dv, _dtype_code(q), eps, _stream(dev))
     else:

@@ -305,9 +305,9 @@ int ret_state_combine(const float* locals, const int* spans, int r, const float*
                                                dk, dv, static_cast<cudaStream_t>(stream)));
 }
 
-int ret_step_gated(const void* q, const void* k, const void* v, const float* gammas,
-                   float* state, const void* gate, void* o, int B, int H, int dk, int dv,
-                   int dtype, float gn_eps, void* stream) {
+int ret_step_rotated(const void* q, const void* k, const void* v, const float* gammas,
+                     const float* theta, long long pos, float* state, const void* gate, void* o,
+                     int B, int H, int dk, int dv, int dtype, float gn_eps, void* stream) {
   if (B < 1 || H < 1 || dk < 8 || dv < 8 || dk % 8 || dv % 8) return RET_EINVAL;
   if (!valid_dtype(dtype)) return RET_EINVAL;
   int s = check_eps(gn_eps);
@@ -317,9 +317,17 @@ int ret_step_gated(const void* q, const void* k, const void* v, const float* gam
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(state) || !aligned16(o))
     return RET_EINVAL;
   if (gate && !aligned16(gate)) return RET_EINVAL;
+  if (theta && (pos < 0 || pos > ((long long)1 << 53))) return RET_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return cuda_status(
-      ret::launch_step(q, k, v, gammas, state, gate, o, B, H, dk, dv, dtype, gn_eps, st));
+  return cuda_status(ret::launch_step(q, k, v, gammas, state, gate, o, B, H, dk, dv, dtype, gn_eps,
+                                      theta, theta ? pos : 0, st));
+}
+
+int ret_step_gated(const void* q, const void* k, const void* v, const float* gammas,
+                   float* state, const void* gate, void* o, int B, int H, int dk, int dv,
+                   int dtype, float gn_eps, void* stream) {
+  return ret_step_rotated(q, k, v, gammas, nullptr, 0, state, gate, o, B, H, dk, dv, dtype,
+                          gn_eps, stream);
 }
 
 int ret_step(const void* q, const void* k, const void* v, const float* gammas, float* state,

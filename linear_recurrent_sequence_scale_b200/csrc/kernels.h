@@ -7,9 +7,11 @@
 namespace ret {
 
 // gate (may be null): o is multiplied by swish(gate), same layout and type as o.
+// theta (may be null): q and k are rotated by pos * theta[c] per channel pair.
 cudaError_t launch_step(const void* q, const void* k, const void* v, const float* gammas,
                         float* state, const void* gate, void* o, int B, int H, int dk, int dv,
-                        int dtype, float eps, cudaStream_t st);
+                        int dtype, float eps, const float* theta, long long pos,
+                        cudaStream_t st);
 
 size_t simt_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk);
 

@@ -15,6 +15,14 @@
 // Consecutive steps on a stream use programmatic dependent launch: a step's
 // CTAs are scheduled while the previous step drains and wait (griddepcontrol)
 // until its writes are visible, which hides the launch gap between steps.
+//
+// Optionally (theta != null) q and k are turned by the xPos rotation of the
+// token's position as they are read ("RetNet - Retentive Network - A
+// Successor to Transformer for LLMs", core components, item 3): channel pair
+// c becomes (x0 cos a - x1 sin a, x0 sin a + x1 cos a), a = pos theta_c, with
+// cos and sin taken in double precision (pos theta reaches 1e6 rad and more).
+// The rotated rows stay in float32 in shared memory; the inputs are not
+// written.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -42,11 +50,12 @@ __device__ __forceinline__ float block_sum_256(float x, float* scratch /* >= 8 f
   return t;
 }
 
-template <typename T, bool GN>
+template <typename T, bool GN, bool ROT>
 __global__ void __launch_bounds__(STEP_THREADS)
 step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
             const float* __restrict__ gammas, float* __restrict__ state,
-            const T* __restrict__ gate, T* __restrict__ o, int H, int dk, int dv, float eps) {
+            const T* __restrict__ gate, T* __restrict__ o, int H, int dk, int dv, float eps,
+            const float* __restrict__ theta, long long pos) {
   extern __shared__ float smem[];
   float* qs = smem;                       // [dk]
   float* ks = smem + dk;                  // [dk]
@@ -65,9 +74,25 @@ step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   const int lane = tid & 31;
   const int rg = tid >> 5;
 
-  for (int i = tid; i < dk; i += STEP_THREADS) {
-    qs[i] = Elem<T>::ld(q + (size_t)bh * dk + i);
-    ks[i] = Elem<T>::ld(k + (size_t)bh * dk + i);
+  if constexpr (ROT) {
+    // dk is even (a multiple of 8): pair c is channels (2c, 2c + 1)
+    for (int c = tid; c < dk / 2; c += STEP_THREADS) {
+      double sn, cs;
+      sincos(static_cast<double>(pos) * static_cast<double>(theta[c]), &sn, &cs);
+      const float fc = static_cast<float>(cs), fs = static_cast<float>(sn);
+      const size_t at = (size_t)bh * dk + 2 * c;
+      const float q0 = Elem<T>::ld(q + at), q1 = Elem<T>::ld(q + at + 1);
+      const float k0 = Elem<T>::ld(k + at), k1 = Elem<T>::ld(k + at + 1);
+      qs[2 * c] = q0 * fc - q1 * fs;
+      qs[2 * c + 1] = q0 * fs + q1 * fc;
+      ks[2 * c] = k0 * fc - k1 * fs;
+      ks[2 * c + 1] = k0 * fs + k1 * fc;
+    }
+  } else {
+    for (int i = tid; i < dk; i += STEP_THREADS) {
+      qs[i] = Elem<T>::ld(q + (size_t)bh * dk + i);
+      ks[i] = Elem<T>::ld(k + (size_t)bh * dk + i);
+    }
   }
   const float g = gammas[h];
   const int c = c0 + 4 * lane;
@@ -149,7 +174,8 @@ step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
 template <typename T>
 static cudaError_t launch_step_t(const void* q, const void* k, const void* v, const float* gammas,
                                  float* state, const void* gate, void* o, int B, int H, int dk,
-                                 int dv, float eps, cudaStream_t st) {
+                                 int dv, float eps, const float* theta, long long pos,
+                                 cudaStream_t st) {
   const int nct = cdiv(dv, STEP_COLS);
   dim3 grid(nct, B * H);
   const size_t smem = sizeof(float) * (2 * dk + STEP_RG * STEP_COLS);
@@ -171,30 +197,31 @@ static cudaError_t launch_step_t(const void* q, const void* k, const void* v, co
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  if (eps < 0.f) {
-    auto fn = step_kernel<T, false>;
+  auto go = [&](auto fn, int nattrs) -> cudaError_t {
     if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      cudaError_t e =
+          cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, fn, qq, kk, vv, gammas, state, gg, oo, H, dk, dv, eps);
-  }
-  auto fn = step_kernel<T, true>;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, fn, qq, kk, vv, gammas, state, gg, oo, H, dk, dv, eps);
+    cfg.numAttrs = nattrs;
+    return cudaLaunchKernelEx(&cfg, fn, qq, kk, vv, gammas, state, gg, oo, H, dk, dv, eps, theta,
+                              pos);
+  };
+  // GroupNorm: the CTAs of one (b, h) form a cluster that exchanges row statistics
+  if (eps < 0.f)
+    return theta ? go(step_kernel<T, false, true>, 1) : go(step_kernel<T, false, false>, 1);
+  return theta ? go(step_kernel<T, true, true>, 2) : go(step_kernel<T, true, false>, 2);
 }
 
 cudaError_t launch_step(const void* q, const void* k, const void* v, const float* gammas,
                         float* state, const void* gate, void* o, int B, int H, int dk, int dv,
-                        int dtype, float eps, cudaStream_t st) {
+                        int dtype, float eps, const float* theta, long long pos,
+                        cudaStream_t st) {
   if (dtype == RET_BF16)
-    return launch_step_t<__nv_bfloat16>(q, k, v, gammas, state, gate, o, B, H, dk, dv, eps, st);
-  return launch_step_t<float>(q, k, v, gammas, state, gate, o, B, H, dk, dv, eps, st);
+    return launch_step_t<__nv_bfloat16>(q, k, v, gammas, state, gate, o, B, H, dk, dv, eps,
+                                        theta, pos, st);
+  return launch_step_t<float>(q, k, v, gammas, state, gate, o, B, H, dk, dv, eps, theta, pos,
+                              st);
 }
 
 }  // namespace ret
