@@ -28,9 +28,11 @@ is needed between steps.  The same line carries:
                 place; % of measured HBM
   cpu_baseline  the float64 CPU oracle on a bounded sample of the same
                 workload (rank 0, N = 1 only)
-With N > 1 (torchrun) every rank runs the same per-GPU step on its own GPU
-(weak scaling, no collective on the data path); the time is the max over
-ranks and `value` counts the tokens of all ranks.
+With --gpus N > 1 the script re-runs itself under torchrun (one process per
+GPU; the driver may also launch it under torchrun directly).  Every rank runs
+the same per-GPU step on its own GPU (weak scaling, no collective on the data
+path); the time is the max over ranks and `value` counts the tokens of all
+ranks.  --plumbing-check runs that launch and aggregation on CPU over gloo.
 
 --impl reference times the CPU oracle (the only reference this build has)
 on a bounded sample of the same workload, on rank 0 only.
@@ -391,253 +393,315 @@ def run_ours(args):
     stream = torch.cuda.current_stream(device)
     launches = 0
 
-    # ---------------- headline: chunkwise on the 6.7B-class layer at 8k ----------------
+    def want(name):
+        return args.only in ("all", name)
+
+    # defaults when the headline is not run (--only <sub-benchmark>)
     w = wl.WORKLOADS[WORKLOAD]
     B, H, N, dk, dv, C, eps = w.B, w.H, w.N, w.dk, w.dv, w.chunk, w.gn_eps
-    if args.batch:
-        B = args.batch  # smaller copy of the workload, for profiler captures only
-    q, k, v, gam = make_qkv(torch, B, H, N, dk, dv, device, seed=1000 + rank)
-    o = torch.empty((B, H, N, dv), dtype=torch.bfloat16, device=device)
-    ws = torch.empty(ret.chunkwise_workspace_bytes(B, H, N, dk, dv, C, torch.bfloat16),
-                     dtype=torch.uint8, device=device)
-    step = lambda: ret.chunkwise(q, k, v, gam, C, gn_eps=eps, out=o, workspace=ws)
-    # the same call in its two phases, so that each kernel's time is measured
-    # live: ret_chunkwise does these two calls on one stream
-    phases = [lambda: ret.chunkwise_states(k, v, gam, C, ws),
-              lambda: ret.chunkwise_output(q, k, v, gam, C, ws, gn_eps=eps, out=o)]
+    value = t_max = roofline = e2e = None
+    headline_launches = 0
     clocks = ClockSampler(smi_index(local))
-    clocks.start()
-    # the step as a user calls it (one ret_chunkwise per step): `value`
-    t_local, t_max = timed(step, args.steps, args.warmup, stream, device)
-    # the same steps split into the two phases with an event between them:
-    # each kernel's duration for the roofline line (the one-call form also
-    # lets the output kernel start while the state scan drains, which the
-    # split run cannot show)
-    _, _, t_phase = timed(step, args.steps, 1, stream, device, phases)
-    clocks.stop()
-    launches += 2 * args.steps  # state scan + chunk output per call
-    headline_launches = launches  # the headline timed region
-    launches += 2 * args.steps    # the phase-split run
-    tokens = B * N
-    value = global_throughput(tokens, args.steps, world, t_max)
-    F = chunkwise_flops(B, H, N, dk, dv, C)
-    F_states, F_out = chunkwise_phase_flops(B, H, N, dk, dv, C)
-    Bytes = chunkwise_bytes(B, H, N, dk, dv)
-    call_s = t_local / args.steps
-    out_s = t_phase[1] / args.steps
-    states_s = t_phase[0] / args.steps
-    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    achieved = F_out / out_s / 1e12
-    traffic = stored_traffic(WORKLOAD)
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic,
-                "kernel": "chunk_out_tc (ret_chunkwise_output), the dominant kernel",
-                "peak_source": f"{peak_src} bf16 burst; sustained "
-                               f"{peaks.get('bf16_tflops_sustained')}",
-                "algorithmic_flop_per_launch": F_out,
-                "kernel_ms": out_s * 1e3,
-                "share_of_step": out_s / (out_s + states_s),
-                "other_kernel": {"name": "state_scan_tc (ret_chunkwise_states)",
-                                 "ms": states_s * 1e3, "algorithmic_flop": F_states,
-                                 "tflops": F_states / states_s / 1e12,
-                                 "frac": F_states / states_s / 1e12 / peak},
-                "whole_call": {"algorithmic_flop": F, "tflops": F / call_s / 1e12,
-                               "frac": F / call_s / 1e12 / peak,
-                               "algorithmic_bytes": Bytes,
-                               "hbm_gbs": Bytes / call_s / 1e9,
-                               "hbm_frac": Bytes / call_s / 1e9 / peaks.get("hbm_gbs", 6650.0)}}
-    del ws
+    if want("headline"):
+        # ---------------- headline: chunkwise on the 6.7B-class layer at 8k ----------------
+        w = wl.WORKLOADS[WORKLOAD]
+        B, H, N, dk, dv, C, eps = w.B, w.H, w.N, w.dk, w.dv, w.chunk, w.gn_eps
+        if args.batch:
+            B = args.batch  # smaller copy of the workload, for profiler captures only
+        q, k, v, gam = make_qkv(torch, B, H, N, dk, dv, device, seed=1000 + rank)
+        o = torch.empty((B, H, N, dv), dtype=torch.bfloat16, device=device)
+        ws = torch.empty(ret.chunkwise_workspace_bytes(B, H, N, dk, dv, C, torch.bfloat16),
+                         dtype=torch.uint8, device=device)
+        step = lambda: ret.chunkwise(q, k, v, gam, C, gn_eps=eps, out=o, workspace=ws)
+        # the same call in its two phases, so that each kernel's time is measured
+        # live: ret_chunkwise does these two calls on one stream
+        phases = [lambda: ret.chunkwise_states(k, v, gam, C, ws),
+                  lambda: ret.chunkwise_output(q, k, v, gam, C, ws, gn_eps=eps, out=o)]
+        clocks = ClockSampler(smi_index(local))
+        clocks.start()
+        # the step as a user calls it (one ret_chunkwise per step): `value`
+        t_local, t_max = timed(step, args.steps, args.warmup, stream, device)
+        # the same steps split into the two phases with an event between them:
+        # each kernel's duration for the roofline line (the one-call form also
+        # lets the output kernel start while the state scan drains, which the
+        # split run cannot show)
+        _, _, t_phase = timed(step, args.steps, 1, stream, device, phases)
+        clocks.stop()
+        launches += 2 * args.steps  # state scan + chunk output per call
+        headline_launches = launches  # the headline timed region
+        launches += 2 * args.steps    # the phase-split run
+        tokens = B * N
+        value = global_throughput(tokens, args.steps, world, t_max)
+        F = chunkwise_flops(B, H, N, dk, dv, C)
+        F_states, F_out = chunkwise_phase_flops(B, H, N, dk, dv, C)
+        Bytes = chunkwise_bytes(B, H, N, dk, dv)
+        call_s = t_local / args.steps
+        out_s = t_phase[1] / args.steps
+        states_s = t_phase[0] / args.steps
+        peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+        achieved = F_out / out_s / 1e12
+        traffic = stored_traffic(WORKLOAD)
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": traffic,
+                    "kernel": "chunk_out_tc (ret_chunkwise_output), the dominant kernel",
+                    "peak_source": f"{peak_src} bf16 burst; sustained "
+                                   f"{peaks.get('bf16_tflops_sustained')}",
+                    "algorithmic_flop_per_launch": F_out,
+                    "kernel_ms": out_s * 1e3,
+                    "share_of_step": out_s / (out_s + states_s),
+                    "other_kernel": {"name": "state_scan_tc (ret_chunkwise_states)",
+                                     "ms": states_s * 1e3, "algorithmic_flop": F_states,
+                                     "tflops": F_states / states_s / 1e12,
+                                     "frac": F_states / states_s / 1e12 / peak},
+                    "whole_call": {"algorithmic_flop": F, "tflops": F / call_s / 1e12,
+                                   "frac": F / call_s / 1e12 / peak,
+                                   "algorithmic_bytes": Bytes,
+                                   "hbm_gbs": Bytes / call_s / 1e9,
+                                   "hbm_frac": Bytes / call_s / 1e9 / peaks.get("hbm_gbs", 6650.0)}}
+        del ws
 
-    # ---------------- e2e through the public API with host buffers ----------------
-    e2e = None
-    if not args.skip_e2e:
-        hq = q.to("cpu").pin_memory()
-        hk = k.to("cpu").pin_memory()
-        hv = v.to("cpu").pin_memory()
-        ho = torch.empty((B, H, N, dv), dtype=torch.bfloat16).pin_memory()
+        # ---------------- e2e through the public API with host buffers ----------------
+        # Every step copies q, k, v from pinned host memory and o back, one
+        # cudaMemcpyAsync per tensor slice.  The batch is cut into slices (one
+        # batch row each) so that the copies of one slice overlap the kernels
+        # of another: host->device on one stream, the retention call on the
+        # compute stream, device->host on a third, ordered by events.
+        e2e = None
+        if not args.skip_e2e:
+            hq = q.to("cpu").pin_memory()
+            hk = k.to("cpu").pin_memory()
+            hv = v.to("cpu").pin_memory()
+            ho = torch.empty((B, H, N, dv), dtype=torch.bfloat16).pin_memory()
+            dq_, dk_, dv_ = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            do_ = torch.empty_like(o)
+            ws1 = torch.empty(ret.chunkwise_workspace_bytes(1, H, N, dk, dv, C, torch.bfloat16),
+                              dtype=torch.uint8, device=device)
+            ws_slices = [ws1, torch.empty_like(ws1)]
+            h2d = torch.cuda.Stream(device)
+            d2h = torch.cuda.Stream(device)
 
-        def e2e_step():
-            dq = hq.to(device, non_blocking=True)
-            dk_ = hk.to(device, non_blocking=True)
-            dv_ = hv.to(device, non_blocking=True)
-            out = ret.chunkwise(dq, dk_, dv_, gam, C, gn_eps=eps)
-            ho.copy_(out, non_blocking=True)
+            def e2e_step():
+                h2d.wait_stream(stream)  # after the previous step (and the start event)
+                for b in range(B):
+                    ev_in = torch.cuda.Event()
+                    with torch.cuda.stream(h2d):
+                        dq_[b].copy_(hq[b], non_blocking=True)
+                        dk_[b].copy_(hk[b], non_blocking=True)
+                        dv_[b].copy_(hv[b], non_blocking=True)
+                        ev_in.record(h2d)
+                    stream.wait_event(ev_in)
+                    ret.chunkwise(dq_[b:b + 1], dk_[b:b + 1], dv_[b:b + 1], gam, C, gn_eps=eps,
+                                  out=do_[b:b + 1], workspace=ws_slices[b & 1])
+                    ev_o = torch.cuda.Event()
+                    ev_o.record(stream)
+                    with torch.cuda.stream(d2h):
+                        d2h.wait_event(ev_o)
+                        ho[b].copy_(do_[b], non_blocking=True)
+                # the step ends when its last output has reached the host
+                stream.wait_stream(d2h)
 
-        e_steps = max(1, min(args.steps, 5))
-        te_local, te_max = timed(e2e_step, e_steps, 1, stream, device)
-        launches += 2 * e_steps
-        e2e = {"value": global_throughput(tokens, e_steps, world, te_max), "unit": "tokens/s",
-               "h2d_bytes_per_step": hq.nbytes + hk.nbytes + hv.nbytes,
-               "d2h_bytes_per_step": ho.nbytes, "steps": e_steps}
-        del hq, hk, hv, ho
-    del q, k, v, o
-    torch.cuda.empty_cache()
+            e_steps = max(3, min(args.steps, 20))
+            te_local, te_max = timed(e2e_step, e_steps, 1, stream, device)
+            launches += 2 * B * e_steps
+            e2e = {"value": global_throughput(tokens, e_steps, world, te_max), "unit": "tokens/s",
+                   "h2d_bytes_per_step": hq.nbytes + hk.nbytes + hv.nbytes,
+                   "d2h_bytes_per_step": ho.nbytes, "steps": e_steps,
+                   "pipeline": f"{B} batch-row slices, copies overlapped with compute"}
+            del hq, hk, hv, ho, dq_, dk_, dv_, do_, ws_slices, ws1
+        del q, k, v, o
+        torch.cuda.empty_cache()
 
     extra = {}
     sub_steps = max(3, min(args.steps, 20))
-    # ---------------- decode ----------------
     if not args.skip_sub:
-        wd = wl.WORKLOADS["decode_6p7b"]
-        qd, kd, vd, gd = make_qkv(torch, wd.B, wd.H, wd.N, wd.dk, wd.dv, device, seed=2000 + rank)
-        s0 = torch.empty((wd.B, wd.H, wd.dk, wd.dv), dtype=torch.float32, device=device)
-        ret.chunkwise(qd, kd, vd, gd, wd.chunk, state_out=s0)  # prefill (untimed)
-        launches += 0
-        del qd, kd, vd
-        states = [s0.clone() for _ in range(4)]
-        T = wl.DECODE_STEPS
-        g = torch.Generator(device=device)
-        g.manual_seed(3000 + rank)
-        sc = 1.0 / math.sqrt(wd.dk)
-        tq = (torch.randn((T, wd.B, wd.H, wd.dk), device=device, generator=g) * sc).bfloat16()
-        tk = (torch.randn((T, wd.B, wd.H, wd.dk), device=device, generator=g) * sc).bfloat16()
-        tv = (torch.randn((T, wd.B, wd.H, wd.dv), device=device, generator=g) * sc).bfloat16()
-        od = torch.empty((wd.B, wd.H, wd.dv), dtype=torch.bfloat16, device=device)
+        # ---------------- decode ----------------
+        if want("decode"):
+            wd = wl.WORKLOADS["decode_6p7b"]
+            qd, kd, vd, gd = make_qkv(torch, wd.B, wd.H, wd.N, wd.dk, wd.dv, device, seed=2000 + rank)
+            s0 = torch.empty((wd.B, wd.H, wd.dk, wd.dv), dtype=torch.float32, device=device)
+            ret.chunkwise(qd, kd, vd, gd, wd.chunk, state_out=s0)  # prefill (untimed)
+            launches += 0
+            del qd, kd, vd
+            states = [s0.clone() for _ in range(4)]
+            T = wl.DECODE_STEPS
+            g = torch.Generator(device=device)
+            g.manual_seed(3000 + rank)
+            sc = 1.0 / math.sqrt(wd.dk)
+            tq = (torch.randn((T, wd.B, wd.H, wd.dk), device=device, generator=g) * sc).bfloat16()
+            tk = (torch.randn((T, wd.B, wd.H, wd.dk), device=device, generator=g) * sc).bfloat16()
+            tv = (torch.randn((T, wd.B, wd.H, wd.dv), device=device, generator=g) * sc).bfloat16()
+            od = torch.empty((wd.B, wd.H, wd.dv), dtype=torch.bfloat16, device=device)
 
-        def decode_run():
-            for t in range(T):
-                ret.step(tq[t], tk[t], tv[t], gd, states[t & 3], out=od)
+            def decode_run():
+                for t in range(T):
+                    ret.step(tq[t], tk[t], tv[t], gd, states[t & 3], out=od)
 
-        td_local, td_max = timed(decode_run, 1, 1, stream, device)
-        launches += T
-        per_step = td_local / T
-        sb = step_bytes(wd.B, wd.H, wd.dk, wd.dv)
-        # the same 1024 steps replayed from a CUDA graph (launch cost hidden)
-        graph_step = None
-        try:
-            gs = torch.cuda.Stream(device)
-            gs.wait_stream(stream)
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.stream(gs):
-                decode_run()  # warm (also sets kernel attributes outside capture)
-                with torch.cuda.graph(graph, stream=gs):
-                    decode_run()
-            stream.wait_stream(gs)
-            tg_local, _ = timed(graph.replay, 1, 1, stream, device)
-            launches += T
-            graph_step = tg_local / T
-            del graph
-        except Exception as ex:  # capture is an optimisation, not a requirement
+            # the 1024-step loop timed REPS times; the median per step is reported
+            REPS = 7
+            plain = [timed(decode_run, 1, 1 if r == 0 else 0, stream, device)[0] / T
+                     for r in range(REPS)]
+            launches += T * REPS
+            per_step = statistics.median(plain)
+            sb = step_bytes(wd.B, wd.H, wd.dk, wd.dv)
+            # the same 1024 steps replayed from a CUDA graph (launch cost hidden)
             graph_step = None
-            extra["decode_graph_error"] = str(ex)[:200]
-        best = min(x for x in (per_step, graph_step) if x is not None)
-        extra["decode"] = {
-            "workload": "decode_6p7b", "steps_per_s": world / max_over_ranks(best, device),
-            "us_per_step": best * 1e6, "us_per_step_launches": per_step * 1e6,
-            "us_per_step_graph": None if graph_step is None else graph_step * 1e6,
-            "tokens_per_s": wd.B * world / max_over_ranks(best, device),
-            "roofline": {"bound": "hbm", "achieved": sb / best / 1e9,
-                         "peak": peaks.get("hbm_gbs", 6650.0), "unit": "GB/s",
-                         "frac": sb / best / 1e9 / peaks.get("hbm_gbs", 6650.0),
-                         "algorithmic_bytes_per_step": sb},
-            "note": "1024 steps over 4 rotating 64 MiB states (working set 256 MiB > L2)"}
-        del states, tq, tk, tv, s0
-        torch.cuda.empty_cache()
+            try:
+                gs = torch.cuda.Stream(device)
+                gs.wait_stream(stream)
+                graph = torch.cuda.CUDAGraph()
+                with torch.cuda.stream(gs):
+                    decode_run()  # warm (also sets kernel attributes outside capture)
+                    with torch.cuda.graph(graph, stream=gs):
+                        decode_run()
+                stream.wait_stream(gs)
+                replays = [timed(graph.replay, 1, 1 if r == 0 else 0, stream, device)[0] / T
+                           for r in range(REPS)]
+                launches += T * REPS
+                graph_step = statistics.median(replays)
+                del graph
+            except Exception as ex:  # capture is an optimisation, not a requirement
+                graph_step = None
+                extra["decode_graph_error"] = str(ex)[:200]
+            best = min(x for x in (per_step, graph_step) if x is not None)
+            extra["decode"] = {
+                "workload": "decode_6p7b", "steps_per_s": world / max_over_ranks(best, device),
+                "us_per_step": best * 1e6, "us_per_step_launches": per_step * 1e6,
+                "us_per_step_graph": None if graph_step is None else graph_step * 1e6,
+                "repetitions": REPS, "statistic": "median of the 1024-step loop timed 7 times",
+                "us_per_step_graph_all": None if graph_step is None else [x * 1e6 for x in replays],
+                "us_per_step_launches_all": [x * 1e6 for x in plain],
+                "tokens_per_s": wd.B * world / max_over_ranks(best, device),
+                "roofline": {"bound": "hbm", "achieved": sb / best / 1e9,
+                             "peak": peaks.get("hbm_gbs", 6650.0), "unit": "GB/s",
+                             "frac": sb / best / 1e9 / peaks.get("hbm_gbs", 6650.0),
+                             "algorithmic_bytes_per_step": sb},
+                "note": "1024 steps over 4 rotating 64 MiB states (working set 256 MiB > L2)"}
+            # the same loop with the xPos rotation of q and k fused into the step
+            # (ret_step_rotated, token positions 8192 + t), plain launches
+            thd = torch.from_numpy(wl.rotation_angles(wd.dk, seed=1)).to(device)
+
+            def decode_run_rot():
+                for t in range(T):
+                    ret.step(tq[t], tk[t], tv[t], gd, states[t & 3], out=od, theta=thd,
+                             pos=wd.N + t)
+
+            rot = [timed(decode_run_rot, 1, 1 if r == 0 else 0, stream, device)[0] / T
+                   for r in range(3)]
+            launches += 3 * T
+            extra["decode"]["rotated_us_per_step_launches"] = statistics.median(rot) * 1e6
+            del states, tq, tk, tv, s0
+            torch.cuda.empty_cache()
 
         # ---------------- parallel form, 1.3B-class layer ----------------
-        wp = wl.WORKLOADS["l1p3b_bf16"]
-        qp, kp, vp, gp = make_qkv(torch, wp.B, wp.H, wp.N, wp.dk, wp.dv, device, seed=4000 + rank)
-        op = torch.empty_like(vp)
-        tpar, _ = timed(lambda: ret.parallel(qp, kp, vp, gp, out=op), sub_steps, 3, stream, device)
-        launches += sub_steps
-        Fp = parallel_flops(wp.B, wp.H, wp.N, wp.dk, wp.dv)
-        cs_ = tpar / sub_steps
-        wsp = torch.empty(ret.chunkwise_workspace_bytes(wp.B, wp.H, wp.N, wp.dk, wp.dv, wp.chunk,
-                                                        torch.bfloat16),
-                          dtype=torch.uint8, device=device)
-        tch, _ = timed(lambda: ret.chunkwise(qp, kp, vp, gp, wp.chunk, out=op, workspace=wsp),
-                       sub_steps, 3, stream, device)
-        launches += 2 * sub_steps
-        Fc = chunkwise_flops(wp.B, wp.H, wp.N, wp.dk, wp.dv, wp.chunk)
-        Bc = chunkwise_bytes(wp.B, wp.H, wp.N, wp.dk, wp.dv)
-        extra["l1p3b"] = {
-            "workload": "l1p3b_bf16",
-            "parallel": {"tokens_per_s": wp.B * wp.N / cs_, "ms": cs_ * 1e3,
-                         "tflops": Fp / cs_ / 1e12, "frac_tc": Fp / cs_ / 1e12 / peak},
-            "chunkwise": {"tokens_per_s": wp.B * wp.N / (tch / sub_steps),
-                          "ms": tch / sub_steps * 1e3,
-                          "tflops": Fc / (tch / sub_steps) / 1e12,
-                          "frac_tc": Fc / (tch / sub_steps) / 1e12 / peak,
-                          "hbm_frac": Bc / (tch / sub_steps) / 1e9 / peaks.get("hbm_gbs", 6650.0)}}
-        del qp, kp, vp, op, wsp
-        torch.cuda.empty_cache()
+        if want("l1p3b"):
+            wp = wl.WORKLOADS["l1p3b_bf16"]
+            qp, kp, vp, gp = make_qkv(torch, wp.B, wp.H, wp.N, wp.dk, wp.dv, device, seed=4000 + rank)
+            op = torch.empty_like(vp)
+            tpar, _ = timed(lambda: ret.parallel(qp, kp, vp, gp, out=op), sub_steps, 3, stream, device)
+            launches += sub_steps
+            Fp = parallel_flops(wp.B, wp.H, wp.N, wp.dk, wp.dv)
+            cs_ = tpar / sub_steps
+            wsp = torch.empty(ret.chunkwise_workspace_bytes(wp.B, wp.H, wp.N, wp.dk, wp.dv, wp.chunk,
+                                                            torch.bfloat16),
+                              dtype=torch.uint8, device=device)
+            tch, _ = timed(lambda: ret.chunkwise(qp, kp, vp, gp, wp.chunk, out=op, workspace=wsp),
+                           sub_steps, 3, stream, device)
+            launches += 2 * sub_steps
+            Fc = chunkwise_flops(wp.B, wp.H, wp.N, wp.dk, wp.dv, wp.chunk)
+            Bc = chunkwise_bytes(wp.B, wp.H, wp.N, wp.dk, wp.dv)
+            extra["l1p3b"] = {
+                "workload": "l1p3b_bf16",
+                "parallel": {"tokens_per_s": wp.B * wp.N / cs_, "ms": cs_ * 1e3,
+                             "tflops": Fp / cs_ / 1e12, "frac_tc": Fp / cs_ / 1e12 / peak},
+                "chunkwise": {"tokens_per_s": wp.B * wp.N / (tch / sub_steps),
+                              "ms": tch / sub_steps * 1e3,
+                              "tflops": Fc / (tch / sub_steps) / 1e12,
+                              "frac_tc": Fc / (tch / sub_steps) / 1e12 / peak,
+                              "hbm_frac": Bc / (tch / sub_steps) / 1e9 / peaks.get("hbm_gbs", 6650.0)}}
+            del qp, kp, vp, op, wsp
+            torch.cuda.empty_cache()
 
         # ---------------- long context 64k ----------------
-        wlg = wl.WORKLOADS["long_64k_bf16"]
-        ql, kl, vl, gl = make_qkv(torch, wlg.B, wlg.H, wlg.N, wlg.dk, wlg.dv, device,
-                                  seed=5000 + rank)
-        ol = torch.empty_like(vl)
-        sl = torch.empty((wlg.B, wlg.H, wlg.dk, wlg.dv), dtype=torch.float32, device=device)
-        wsl = torch.empty(ret.chunkwise_workspace_bytes(wlg.B, wlg.H, wlg.N, wlg.dk, wlg.dv,
-                                                        wlg.chunk, torch.bfloat16),
-                          dtype=torch.uint8, device=device)
-        tl, _ = timed(lambda: ret.chunkwise(ql, kl, vl, gl, wlg.chunk, out=ol, state_out=sl,
-                                            workspace=wsl), sub_steps, 3, stream, device)
-        launches += 2 * sub_steps
-        Fl = chunkwise_flops(wlg.B, wlg.H, wlg.N, wlg.dk, wlg.dv, wlg.chunk, state_out=True)
-        cl = tl / sub_steps
-        extra["long_64k"] = {"workload": "long_64k_bf16", "tokens_per_s": wlg.N / cl,
-                             "ms": cl * 1e3, "tflops": Fl / cl / 1e12,
-                             "frac_tc": Fl / cl / 1e12 / peak}
-        del ql, kl, vl, ol, sl, wsl
-        torch.cuda.empty_cache()
+        if want("long_64k"):
+            wlg = wl.WORKLOADS["long_64k_bf16"]
+            ql, kl, vl, gl = make_qkv(torch, wlg.B, wlg.H, wlg.N, wlg.dk, wlg.dv, device,
+                                      seed=5000 + rank)
+            ol = torch.empty_like(vl)
+            sl = torch.empty((wlg.B, wlg.H, wlg.dk, wlg.dv), dtype=torch.float32, device=device)
+            wsl = torch.empty(ret.chunkwise_workspace_bytes(wlg.B, wlg.H, wlg.N, wlg.dk, wlg.dv,
+                                                            wlg.chunk, torch.bfloat16),
+                              dtype=torch.uint8, device=device)
+            tl, _ = timed(lambda: ret.chunkwise(ql, kl, vl, gl, wlg.chunk, out=ol, state_out=sl,
+                                                workspace=wsl), sub_steps, 3, stream, device)
+            launches += 2 * sub_steps
+            Fl = chunkwise_flops(wlg.B, wlg.H, wlg.N, wlg.dk, wlg.dv, wlg.chunk, state_out=True)
+            cl = tl / sub_steps
+            extra["long_64k"] = {"workload": "long_64k_bf16", "tokens_per_s": wlg.N / cl,
+                                 "ms": cl * 1e3, "tflops": Fl / cl / 1e12,
+                                 "frac_tc": Fl / cl / 1e12 / peak}
+            del ql, kl, vl, ol, sl, wsl
+            torch.cuda.empty_cache()
 
         # ---------------- backward on the 1.3B-class layer ----------------
-        wb = wl.WORKLOADS["l1p3b_bf16"]
-        qb, kb, vb, gb = make_qkv(torch, wb.B, wb.H, wb.N, wb.dk, wb.dv, device, seed=7000 + rank)
-        dob = (torch.randn(vb.shape, device=device) * 0.1).bfloat16()
-        wsb = torch.empty(ret.load_library().ret_chunkwise_backward_workspace(
-            wb.B, wb.H, wb.N, wb.dk, wb.dv, wb.chunk, ret.RET_BF16), dtype=torch.uint8,
-            device=device)
-        tb, _ = timed(lambda: ret.chunkwise_backward(qb, kb, vb, gb, wb.chunk, dob, workspace=wsb),
-                      3, 1, stream, device)
-        launches += 3 * 7   # two state scans, two score and three gradient products
-        Fb = 2 * chunkwise_flops(wb.B, wb.H, wb.N, wb.dk, wb.dv, wb.chunk)
-        cb = tb / 3
-        extra["backward"] = {"workload": "l1p3b_bf16 chunkwise backward (dq, dk, dv)",
-                             "ms": cb * 1e3, "tokens_per_s": wb.B * wb.N / cb,
-                             "tflops": Fb / cb / 1e12,
-                             "note": "CUDA cores, float32; flops counted as twice the forward's"}
-        del qb, kb, vb, dob, wsb
-        torch.cuda.empty_cache()
+        if want("backward"):
+            wb = wl.WORKLOADS["l1p3b_bf16"]
+            qb, kb, vb, gb = make_qkv(torch, wb.B, wb.H, wb.N, wb.dk, wb.dv, device, seed=7000 + rank)
+            dob = (torch.randn(vb.shape, device=device) * 0.1).bfloat16()
+            wsb = torch.empty(ret.load_library().ret_chunkwise_backward_workspace(
+                wb.B, wb.H, wb.N, wb.dk, wb.dv, wb.chunk, ret.RET_BF16), dtype=torch.uint8,
+                device=device)
+            tb, _ = timed(lambda: ret.chunkwise_backward(qb, kb, vb, gb, wb.chunk, dob, workspace=wsb),
+                          3, 1, stream, device)
+            launches += 3 * 7   # two state scans, two score and three gradient products
+            Fb = 2 * chunkwise_flops(wb.B, wb.H, wb.N, wb.dk, wb.dv, wb.chunk)
+            cb = tb / 3
+            extra["backward"] = {"workload": "l1p3b_bf16 chunkwise backward (dq, dk, dv)",
+                                 "ms": cb * 1e3, "tokens_per_s": wb.B * wb.N / cb,
+                                 "tflops": Fb / cb / 1e12,
+                                 "note": "CUDA cores, float32; flops counted as twice the forward's"}
+            del qb, kb, vb, dob, wsb
+            torch.cuda.empty_cache()
 
         # ---------------- xPos rotation of q and k, 6.7B-class 8k layer ----------------
-        wr = wl.WORKLOADS["l6p7b_8k_bf16"]
-        qr, kr, vr, _ = make_qkv(torch, wr.B, wr.H, wr.N, wr.dk, wr.dv, device, seed=8000 + rank)
-        del vr
-        thr = torch.from_numpy(wl.rotation_angles(wr.dk, seed=1)).to(device)
-        tr, _ = timed(lambda: (ret.rotate(qr, thr, 0, out=qr), ret.rotate(kr, thr, 0, out=kr)),
-                      sub_steps, 3, stream, device)
-        launches += 2 * sub_steps
-        Br = 2 * 2 * qr.numel() * qr.element_size()   # q and k, each read and written once
-        cr = tr / sub_steps
-        extra["rotate"] = {"workload": "l6p7b_8k_bf16 xPos rotation of q and k, in place",
-                           "ms": cr * 1e3, "hbm_gbs": Br / cr / 1e9,
-                           "hbm_frac": Br / cr / 1e9 / peaks.get("hbm_gbs", 6650.0)}
-        del qr, kr
-        torch.cuda.empty_cache()
+        if want("rotate"):
+            wr = wl.WORKLOADS["l6p7b_8k_bf16"]
+            qr, kr, vr, _ = make_qkv(torch, wr.B, wr.H, wr.N, wr.dk, wr.dv, device, seed=8000 + rank)
+            del vr
+            thr = torch.from_numpy(wl.rotation_angles(wr.dk, seed=1)).to(device)
+            tr, _ = timed(lambda: (ret.rotate(qr, thr, 0, out=qr), ret.rotate(kr, thr, 0, out=kr)),
+                          sub_steps, 3, stream, device)
+            launches += 2 * sub_steps
+            Br = 2 * 2 * qr.numel() * qr.element_size()   # q and k, each read and written once
+            cr = tr / sub_steps
+            extra["rotate"] = {"workload": "l6p7b_8k_bf16 xPos rotation of q and k, in place",
+                               "ms": cr * 1e3, "hbm_gbs": Br / cr / 1e9,
+                               "hbm_frac": Br / cr / 1e9 / peaks.get("hbm_gbs", 6650.0)}
+            del qr, kr
+            torch.cuda.empty_cache()
 
         # ---------------- gated output on the headline workload ----------------
-        qg, kg, vg, gg = make_qkv(torch, w.B, w.H, w.N, w.dk, w.dv, device, seed=6000 + rank)
-        gate = torch.randn(vg.shape, device=device).bfloat16()
-        og = torch.empty_like(vg)
-        wsg = torch.empty(ret.chunkwise_workspace_bytes(w.B, w.H, w.N, w.dk, w.dv, w.chunk,
-                                                        torch.bfloat16),
-                          dtype=torch.uint8, device=device)
-        tg, _ = timed(lambda: ret.chunkwise(qg, kg, vg, gg, w.chunk, gn_eps=w.gn_eps, out=og,
-                                            workspace=wsg, gate=gate),
-                      sub_steps, 3, stream, device)
-        tu, _ = timed(lambda: ret.chunkwise(qg, kg, vg, gg, w.chunk, gn_eps=w.gn_eps, out=og,
-                                            workspace=wsg),
-                      sub_steps, 3, stream, device)
-        launches += 4 * sub_steps
-        cg_ = tg / sub_steps
-        extra["gated"] = {"workload": WORKLOAD + " with swish(gate) * GroupNorm(o)",
-                          "tokens_per_s": w.B * w.N / cg_, "ms": cg_ * 1e3,
-                          "ungated_ms": tu / sub_steps * 1e3,
-                          "tflops": F / cg_ / 1e12, "frac_tc": F / cg_ / 1e12 / peak,
-                          "gate_bytes": gate.numel() * gate.element_size()}
-        del qg, kg, vg, og, wsg, gate
-        torch.cuda.empty_cache()
+        if want("gated"):
+            qg, kg, vg, gg = make_qkv(torch, w.B, w.H, w.N, w.dk, w.dv, device, seed=6000 + rank)
+            gate = torch.randn(vg.shape, device=device).bfloat16()
+            og = torch.empty_like(vg)
+            wsg = torch.empty(ret.chunkwise_workspace_bytes(w.B, w.H, w.N, w.dk, w.dv, w.chunk,
+                                                            torch.bfloat16),
+                              dtype=torch.uint8, device=device)
+            tg, _ = timed(lambda: ret.chunkwise(qg, kg, vg, gg, w.chunk, gn_eps=w.gn_eps, out=og,
+                                                workspace=wsg, gate=gate),
+                          sub_steps, 3, stream, device)
+            tu, _ = timed(lambda: ret.chunkwise(qg, kg, vg, gg, w.chunk, gn_eps=w.gn_eps, out=og,
+                                                workspace=wsg),
+                          sub_steps, 3, stream, device)
+            launches += 4 * sub_steps
+            cg_ = tg / sub_steps
+            extra["gated"] = {"workload": WORKLOAD + " with swish(gate) * GroupNorm(o)",
+                              "tokens_per_s": w.B * w.N / cg_, "ms": cg_ * 1e3,
+                              "ungated_ms": tu / sub_steps * 1e3,
+                              "tflops": F / cg_ / 1e12, "frac_tc": F / cg_ / 1e12 / peak,
+                              "gate_bytes": gate.numel() * gate.element_size()}
+            del qg, kg, vg, og, wsg, gate
+            torch.cuda.empty_cache()
 
     # ---------------- CPU oracle baseline ----------------
     cpu = None
@@ -652,7 +716,8 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": t_max / args.steps * 1e3, "higher_is_better": True,
+            "ms_per_step": None if t_max is None else t_max / args.steps * 1e3,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": WORKLOAD if not args.batch else f"{WORKLOAD} (batch {B})",
                        "global_batch": B * world, "seq_len": N, "heads": H,
@@ -668,9 +733,49 @@ def run_ours(args):
     return 0
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def rank_launch_command(gpus: int, argv, port: int):
+    """The torchrun command that runs this script once per GPU (one process
+    per GPU, rendezvous on 127.0.0.1)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__), *argv]
+
+
+def launch_ranks(gpus: int, argv) -> int:
+    """Re-run this script under torchrun with `gpus` ranks; rank 0 prints the
+    line.  Used when --gpus N > 1 is given outside torchrun."""
+    return subprocess.call(rank_launch_command(gpus, argv, free_port()))
+
+
+def run_plumbing_check(args):
+    """The multi-rank plumbing without a GPU: every rank joins a gloo group,
+    reports a fixed per-rank time (rank r takes 0.5 + r seconds for `steps`
+    steps of the headline's tokens) and rank 0 prints n_gpus, the max time
+    and the whole-job throughput, exactly as the GPU run aggregates them."""
+    rank, world = init_dist("gloo")
+    from linear_recurrent_sequence_scale_b200 import workloads as wl
+    w = wl.WORKLOADS[WORKLOAD]
+    t_local = 0.5 + rank
+    barrier()
+    t_max = max_over_ranks(t_local)
+    value = global_throughput(w.B * w.N, args.steps, world, t_max)
+    if rank == 0:
+        print(json.dumps({"plumbing_check": True, "n_gpus": world, "gpus_requested": args.gpus,
+                          "t_max_s": t_max, "value": value, "unit": "tokens/s"}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="GPUs (ranks); outside torchrun, N > 1 re-runs this script under it")
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
@@ -679,11 +784,33 @@ def main(argv=None):
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-sub", action="store_true", help="headline only")
+    ap.add_argument("--only", default="all",
+                    choices=["all", "headline", "decode", "l1p3b", "long_64k", "backward", "rotate",
+                             "gated"],
+                    help="run one part (profiler captures); the line then lacks the others")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the headline batch (smaller profiler captures only)")
-    args = ap.parse_args(argv)
+    ap.add_argument("--plumbing-check", action="store_true",
+                    help="CPU only: run the rank launch and the cross-rank aggregation over gloo, "
+                         "no kernels")
+    raw = list(sys.argv[1:] if argv is None else argv)
+    args = ap.parse_args(raw)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_ranks(args.gpus, raw)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus:
+        ap.error(f"--gpus {args.gpus} but {world} ranks were launched")
+    if args.plumbing_check:
+        try:
+            return run_plumbing_check(args)
+        finally:
+            import torch.distributed as dist
+            if dist.is_initialized():
+                dist.destroy_process_group()
     if args.impl == "reference":
         return run_reference(args)
     try:

@@ -79,3 +79,31 @@ def test_two_ranks_take_the_max_time_and_sum_the_tokens():
     t_max, value = out[0]
     assert t_max == pytest.approx(1.5)
     assert value == pytest.approx(65536 * 10 * 2 / 1.5)
+
+
+def test_gpus_flag_launches_that_many_ranks_and_sums_their_tokens():
+    """`bench.py --gpus 2` outside torchrun re-runs itself as two ranks; rank 0
+    prints n_gpus = 2, the max time over the ranks and both ranks' tokens."""
+    import json
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--steps", "10", "--warmup", "3", "--plumbing-check"],
+                       capture_output=True, text=True, timeout=240, env=env, cwd=root)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(x) for x in r.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1, r.stdout          # rank 0 alone prints
+    line = lines[0]
+    assert line["n_gpus"] == 2 and line["gpus_requested"] == 2
+    assert line["t_max_s"] == pytest.approx(1.5)
+    assert line["value"] == pytest.approx(8 * 8192 * 10 * 2 / 1.5)
+
+
+def test_rank_launch_command_uses_torchrun_on_loopback():
+    cmd = bench.rank_launch_command(4, ["--gpus", "4", "--steps", "5"], 29555)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd
+    assert "--master-port=29555" in cmd and cmd[-4:] == ["--gpus", "4", "--steps", "5"]
