@@ -69,7 +69,7 @@ struct Params {
   int write_ws0;      // store state_in (as bf16) in slot 0
 };
 
-template <bool SPLIT>
+template <bool SPLIT, int MH>
 __global__ void __launch_bounds__(THREADS, 1)
 state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const Params p) {
@@ -151,6 +151,13 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, p.nt, true, true);
+      // descriptors of ring slot 0, built once; a slot, a d_k half or a
+      // 16-token step is a constant offset of the start address (low bits,
+      // 16-byte units), so the issue loop does no descriptor arithmetic
+      const uint32_t s0 = smem_u32(smem);
+      const uint64_t a0 = sdesc_sw128(s0 + K_OFF, BOX, 1024);
+      const uint64_t bh0 = sdesc_sw128(s0 + V_OFF, BOX, 1024);
+      const uint64_t bl0 = sdesc_sw128(s0 + LO_OFF, BOX, 1024);
       int g = 0;
       bool ok = true;
       for (int ci = 0; ci < p.nc && ok; ++ci) {
@@ -163,16 +170,16 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
           const int slot = g % STAGES;
           if (!mbar_wait(&xf[slot], (g / STAGES) & 1, 103)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t sb = smem_u32(smem + slot * STAGE_BYTES);
+          const uint64_t so = static_cast<uint64_t>((slot * STAGE_BYTES) >> 4);
 #pragma unroll
           for (int kk = 0; kk < T / 16; ++kk) {
-            const uint64_t bhi = sdesc_sw128(sb + V_OFF + kk * 2048, BOX, 1024);
-            const uint64_t blo = sdesc_sw128(sb + LO_OFF + kk * 2048, BOX, 1024);
-            for (int hh = 0; hh < p.mh; ++hh) {
-              const uint64_t a = sdesc_sw128(sb + K_OFF + 2 * hh * BOX + kk * 2048, BOX, 1024);
+            const uint64_t ko = so + ((kk * 2048) >> 4);
+#pragma unroll
+            for (int hh = 0; hh < MH; ++hh) {
+              const uint64_t a = a0 + ko + ((2 * hh * BOX) >> 4);
               const uint32_t d = tmem + hh * p.nt;
-              umma_bf16_ss(d, a, bhi, idesc, first ? 0u : 1u);
-              if (SPLIT) umma_bf16_ss(d, a, blo, idesc, 1u);
+              umma_bf16_ss(d, a, bh0 + ko, idesc, first ? 0u : 1u);
+              if (SPLIT) umma_bf16_ss(d, a, bl0 + ko, idesc, 1u);
             }
             first = false;
           }
@@ -293,14 +300,12 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       tc_fence_after();
       const float gL = gpow(lg, min(p.chunk, p.N - ci * p.chunk));
       const bool last = ci == p.nc - 1;
-      // R <- gamma^L R + H, 32 columns at a time; the MMA warp reuses H for the
-      // next chunk only after every thread has read it (h_free).  This kernel
-      // is bound by its loads, not by the tensor core, so that wait is cheap.
+      // R <- gamma^L R + H, 32 columns at a time, in TMEM only; H goes back to
+      // the MMA warp (h_free) as soon as it has been read, and the stores of
+      // the new state to global memory follow from TMEM, off that path.
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         if (hh >= p.mh) continue;
-        const int r = r0 + 128 * hh + row;
-        const bool live = r < p.dk;
 #pragma unroll
         for (int x0 = 0; x0 < 64; x0 += 32) {
           if (x0 >= ncol) continue;
@@ -312,7 +317,25 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 #pragma unroll
           for (int x = 0; x < 32; ++x)
             v[x] = __float_as_uint(fmaf(gL, __uint_as_float(v[x]), __uint_as_float(hv[x])));
-          if (!last) tmem_st32(tmem + rcol + hoff, v);
+          tmem_st32(tmem + rcol + hoff, v);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(h_free);
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        if (hh >= p.mh) continue;
+        const int r = r0 + 128 * hh + row;
+        const bool live = r < p.dk;
+#pragma unroll
+        for (int x0 = 0; x0 < 64; x0 += 32) {
+          if (x0 >= ncol) continue;
+          const uint32_t hoff = lane_addr + hh * p.nt + part * ncol + x0;
+          uint32_t v[32];
+          tmem_ld32(tmem + rcol + hoff, v);  // warp-wide: every lane loads
+          tmem_wait_ld();
           if (!live) continue;
           if (!last) {
             uint4* dst = reinterpret_cast<uint4*>(
@@ -334,10 +357,6 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
           }
         }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(h_free);
     }
   }
 
@@ -384,18 +403,15 @@ cudaError_t launch_tc_state(const void* k, const void* v, const float* gammas, i
   const int halves = cdiv(dk, 128);
   p.mh = (halves == 2 && BH * (uint64_t)(dv / p.nt) >= (uint64_t)nsm) ? 2 : 1;
   dim3 grid(dv / p.nt, halves / p.mh, (unsigned)BH);
-  if (state_out) {
-    auto fn = state_scan_tc<true>;
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+  auto go = [&](auto fn) -> cudaError_t {
+    cudaError_t e2 = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          SMEM_BYTES);
+    if (e2 != cudaSuccess) return e2;
     fn<<<grid, THREADS, SMEM_BYTES, st>>>(tm_k, tm_v, p);
-  } else {
-    auto fn = state_scan_tc<false>;
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    fn<<<grid, THREADS, SMEM_BYTES, st>>>(tm_k, tm_v, p);
-  }
-  return cudaPeekAtLastError();
+    return cudaPeekAtLastError();
+  };
+  if (state_out) return p.mh == 2 ? go(state_scan_tc<true, 2>) : go(state_scan_tc<true, 1>);
+  return p.mh == 2 ? go(state_scan_tc<false, 2>) : go(state_scan_tc<false, 1>);
 }
 
 }  // namespace ret
