@@ -39,14 +39,21 @@ using namespace sm100;
 constexpr int T = 64;                  // tokens per stage (32 measured slower: more
                                        // per-stage waits and fences per token)
 constexpr int NT = 128;                // state columns per CTA (d_v = 64 uses 64)
-constexpr int STAGES = 3;              // 3 x 64 KB
 constexpr int BOX = T * 128;           // one [T][64] bf16 box
 constexpr int K_OFF = 0;               // 4 boxes: up to 256 rows of d_k
 constexpr int V_OFF = 4 * BOX;         // 2 boxes: NT columns of V, becomes V hi
-constexpr int LO_OFF = 6 * BOX;        // 2 boxes
-constexpr int STAGE_BYTES = 8 * BOX;
-constexpr int BAR_OFF = STAGES * STAGE_BYTES;
-constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;
+constexpr int LO_OFF = 6 * BOX;        // 2 boxes (V lo, with the hi/lo split only)
+// Ring geometry: with the hi/lo split a stage holds K, V hi and V lo (64 KB,
+// 3 stages); without it K and V (48 KB), and the same shared memory holds 4
+// stages, so more loads are in flight behind the transform and the MMAs.
+template <bool SPLIT> struct Ring {
+  static constexpr int STAGES = SPLIT ? 3 : 4;
+  static constexpr int STAGE_BYTES = (SPLIT ? 8 : 6) * BOX;
+  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
+};
+constexpr int SMEM_BYTES = 3 * 8 * BOX + 512 + 1024;
+static_assert(Ring<true>::BAR_OFF + 512 + 1024 <= SMEM_BYTES &&
+              Ring<false>::BAR_OFF + 512 + 1024 <= SMEM_BYTES, "ring fits");
 constexpr int XF_WARPS = 8;            // V (.) zeta warps
 #ifndef RET_K2_XG
 #define RET_K2_XG 1
@@ -56,7 +63,9 @@ constexpr int XG_THREADS = XF_WARPS * 32 / XG;
 // Each ring slot must belong to one group, so that a group waiting on a
 // slot's mbarrier is never more than one phase ahead of it (a parity wait
 // two phases ahead would pass at once).
-static_assert(XF_WARPS % XG == 0 && STAGES % XG == 0, "transform groups own whole ring slots");
+static_assert(XF_WARPS % XG == 0 && Ring<true>::STAGES % XG == 0 &&
+                  Ring<false>::STAGES % XG == 0,
+              "transform groups own whole ring slots");
 constexpr int EPI_WARP0 = 2 + XF_WARPS;  // first state warp
 constexpr int THREADS = (EPI_WARP0 + 8) * 32;  // 18 warps
 
@@ -76,6 +85,9 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
+  constexpr int STAGES = Ring<SPLIT>::STAGES;
+  constexpr int STAGE_BYTES = Ring<SPLIT>::STAGE_BYTES;
+  constexpr int BAR_OFF = Ring<SPLIT>::BAR_OFF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
   uint64_t* full = bars;                 // TMA -> transform
   uint64_t* xf = bars + STAGES;          // transform -> MMA
