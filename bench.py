@@ -443,13 +443,13 @@ def run_ours(args):
         traffic = stored_traffic(WORKLOAD)
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": traffic,
-                    "kernel": "chunk_out_tc (ret_chunkwise_output), the dominant kernel",
+                    "kernel": "k3::chunk_out_tc (ret_chunkwise_output), the dominant kernel",
                     "peak_source": f"{peak_src} bf16 burst; sustained "
                                    f"{peaks.get('bf16_tflops_sustained')}",
                     "algorithmic_flop_per_launch": F_out,
                     "kernel_ms": out_s * 1e3,
                     "share_of_step": out_s / (out_s + states_s),
-                    "other_kernel": {"name": "state_scan_tc (ret_chunkwise_states)",
+                    "other_kernel": {"name": "k2::state_scan_tc (ret_chunkwise_states)",
                                      "ms": states_s * 1e3, "algorithmic_flop": F_states,
                                      "tflops": F_states / states_s / 1e12,
                                      "frac": F_states / states_s / 1e12 / peak},
@@ -607,8 +607,15 @@ def run_ours(args):
             tch, _ = timed(lambda: ret.chunkwise(qp, kp, vp, gp, wp.chunk, out=op, workspace=wsp),
                            sub_steps, 3, stream, device)
             launches += 2 * sub_steps
+            # the same call split into its two kernels, each timed live
+            _, _, tph = timed(None, sub_steps, 0, stream, device,
+                              [lambda: ret.chunkwise_states(kp, vp, gp, wp.chunk, wsp),
+                               lambda: ret.chunkwise_output(qp, kp, vp, gp, wp.chunk, wsp,
+                                                            out=op)])
+            launches += 2 * sub_steps
             Fc = chunkwise_flops(wp.B, wp.H, wp.N, wp.dk, wp.dv, wp.chunk)
             Bc = chunkwise_bytes(wp.B, wp.H, wp.N, wp.dk, wp.dv)
+            Fcs, Fco = chunkwise_phase_flops(wp.B, wp.H, wp.N, wp.dk, wp.dv, wp.chunk)
             extra["l1p3b"] = {
                 "workload": "l1p3b_bf16",
                 "parallel": {"tokens_per_s": wp.B * wp.N / cs_, "ms": cs_ * 1e3,
@@ -617,7 +624,11 @@ def run_ours(args):
                               "ms": tch / sub_steps * 1e3,
                               "tflops": Fc / (tch / sub_steps) / 1e12,
                               "frac_tc": Fc / (tch / sub_steps) / 1e12 / peak,
-                              "hbm_frac": Bc / (tch / sub_steps) / 1e9 / peaks.get("hbm_gbs", 6650.0)}}
+                              "hbm_frac": Bc / (tch / sub_steps) / 1e9 / peaks.get("hbm_gbs", 6650.0),
+                              "states_ms": tph[0] / sub_steps * 1e3,
+                              "output_ms": tph[1] / sub_steps * 1e3,
+                              "states_tflops": Fcs / (tph[0] / sub_steps) / 1e12,
+                              "output_tflops": Fco / (tph[1] / sub_steps) / 1e12}}
             del qp, kp, vp, op, wsp
             torch.cuda.empty_cache()
 
@@ -652,13 +663,17 @@ def run_ours(args):
                 device=device)
             tb, _ = timed(lambda: ret.chunkwise_backward(qb, kb, vb, gb, wb.chunk, dob, workspace=wsb),
                           3, 1, stream, device)
-            launches += 3 * 7   # two state scans, two score and three gradient products
+            # bf16: six row reversals, three forward calls of two kernels each and
+            # the d state_in scaling
+            launches += 3 * 13
             Fb = 2 * chunkwise_flops(wb.B, wb.H, wb.N, wb.dk, wb.dv, wb.chunk)
             cb = tb / 3
             extra["backward"] = {"workload": "l1p3b_bf16 chunkwise backward (dq, dk, dv)",
                                  "ms": cb * 1e3, "tokens_per_s": wb.B * wb.N / cb,
                                  "tflops": Fb / cb / 1e12,
-                                 "note": "CUDA cores, float32; flops counted as twice the forward's"}
+                                 "note": "bf16: three forward chunkwise calls of permuted and "
+                                         "row-reversed inputs on the tensor cores; flops counted "
+                                         "as twice the forward's"}
             del qb, kb, vb, dob, wsb
             torch.cuda.empty_cache()
 

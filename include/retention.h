@@ -37,7 +37,10 @@
  *    that nothing was launched and no memory was written.  Errors raised by a
  *    kernel while it runs surface on the stream like any CUDA error.
  *  - Accumulation is float32.  With RET_BF16 inputs the products run on the
- *    tensor cores with bf16 operands; o is rounded to the input type.
+ *    tensor cores with bf16 operands where the shapes fit their tiles (the
+ *    rules under each call); other bf16 shapes (chunk 64, dk 32, dk 512 ...)
+ *    run the float32 CUDA-core kernels on the same inputs, whose only bf16
+ *    rounding is that of o.  Either way o is rounded to the input type.
  */
 #ifndef RETENTION_H_
 #define RETENTION_H_
@@ -95,8 +98,9 @@ RET_API size_t ret_chunkwise_workspace(int B, int H, int N, int dk, int dv, int 
  *                its contents on entry do not matter; it is overwritten.
  * The final state is accurate to float32 accumulation (the bf16 path splits
  * the decayed V operand into two bf16 halves when state_out is requested).
- * Supported: chunk >= 1 with RET_F32; chunk in {128, 256, 512} for the tensor
- * core path of RET_BF16, under the same dk/dv rules as ret_parallel.
+ * Supported: chunk >= 1 with either type.  RET_BF16 runs on the tensor cores
+ * for chunk in {128, 256, 512} under the dk/dv rules of ret_parallel, and on
+ * the float32 CUDA-core kernels otherwise (chunk 64, for instance).
  */
 RET_API int ret_chunkwise(const void* q, const void* k, const void* v, const float* gammas, int chunk,
                   const float* state_in, float* state_out, void* o,

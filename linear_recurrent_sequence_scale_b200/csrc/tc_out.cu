@@ -14,13 +14,9 @@
 // and overlaps consecutive tiles:
 //   warp 0     TMA: Q of the next tile into the second of two Q buffers while
 //              the current tile runs; K, V and R_{i-1} tiles through a 3-stage
-//              ring of 32 KB stages, in the order the MMAs consume them (V and
-//              R in 16 KB boxes of 128 rows: one stage is 128 keys or 128 rows
-//              of d_k by a 128-column half of the slice, since a producer
-//              iteration costs about the same whatever its bytes)
+//              ring of 32 KB stages, in the order the MMAs consume them
 //   warp 1     tcgen05.mma: S_t = Q K_t^T into one of two 128-column TMEM
 //              buffers; O += P_t V_t with P_t read from TMEM; O += (Q (.) xi) R
-//              (P V and the cross term as N = 128 MMAs per column half)
 //   warps 2-5  decay mask: S_t -> registers -> P_t = S_t (.) D as bf16, written
 //              back into the first 64 columns of S_t's TMEM buffer; then
 //              Q (.) xi in place in the tile's Q buffer
@@ -56,6 +52,7 @@ constexpr int BN = 128;                // keys per key tile
 constexpr int DVS = 256;               // output columns per CTA
 constexpr int STAGE = 32768;
 constexpr int QBOX = 128 * 128;        // [128 rows][64] bf16 = 16 KB
+constexpr int VBOX = 64 * 128;         // [64 rows][64] bf16 = 8 KB
 constexpr int QBUF = 4 * QBOX;         // one Q tile, d_k <= 256
 constexpr int Q_OFF = 0;
 constexpr int DATA_BYTES = 7 * 32768;  // Q buffers + ring stages
@@ -228,10 +225,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
   constexpr int kq = KQ;              // 64-wide blocks of d_k
   constexpr int kst = (KQ + 1) / 2;   // K-tile stages (two blocks each)
   constexpr int KST = kst;
-  const int chw = p.dvs < 128 ? p.dvs : 128;  // columns per V / R stage (a column half)
-  const int nch = p.dvs / chw;                 // column halves of the slice
-  const int hb = chw / 64;                     // 64-wide boxes per stage
-  const int rrows = p.dk < 128 ? p.dk : 128;   // d_k rows per R stage
+  const int vb = p.dvs / 64;          // 64-wide blocks of the column slice
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
   uint64_t* full = bars;              // [RING]
@@ -341,12 +335,12 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
           }
           if (t >= 1 && ok) {
             const int key0 = x.cs + (t - 1) * BN;
-            for (int c = 0; c < nch && ok; ++c, ++g) {
+            for (int s = 0; s < 2 && ok; ++s, ++g) {
               uint64_t* bar;
-              uint8_t* st = acquire(hb * QBOX, bar);
+              uint8_t* st = acquire(vb * VBOX, bar);
               if (!st) { ok = false; break; }
-              for (int b = 0; b < hb; ++b)
-                tma_load_3d(st + b * QBOX, &tm_v, bar, c0 + c * chw + b * 64, key0, x.bh);
+              for (int b = 0; b < vb; ++b)
+                tma_load_3d(st + b * VBOX, &tm_v, bar, c0 + b * 64, key0 + 64 * s, x.bh);
             }
           }
         }
@@ -359,14 +353,12 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             r_ready = true;
           }
           const int zr = x.bh * p.nc + x.ci;
-          for (int dh = 0; dh < p.dk / rrows && ok; ++dh) {
-            for (int c = 0; c < nch && ok; ++c, ++g) {
-              uint64_t* bar;
-              uint8_t* st = acquire(hb * rrows * 128, bar);
-              if (!st) { ok = false; break; }
-              for (int b = 0; b < hb; ++b)
-                tma_load_3d(st + b * rrows * 128, &tm_r, bar, c0 + c * chw + b * 64, dh * rrows, zr);
-            }
+          for (int s = 0; s < kq && ok; ++s, ++g) {
+            uint64_t* bar;
+            uint8_t* st = acquire(vb * VBOX, bar);
+            if (!st) { ok = false; break; }
+            for (int b = 0; b < vb; ++b)
+              tma_load_3d(st + b * VBOX, &tm_r, bar, c0 + b * 64, 64 * s, zr);
           }
         }
       }
@@ -378,7 +370,7 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t id_qk = idesc_bf16(128, BN, false, false);
-      const uint32_t id_pv = idesc_bf16(128, chw, false, true);
+      const uint32_t id_pv = idesc_bf16(128, p.dvs, false, true);
       const uint32_t o_tm = tmem + 256;
       int g = 0, sc = 0, k = 0;
       bool ok = true;
@@ -436,14 +428,15 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
             tc_fence_after();
             const uint32_t pa = tmem + b * BN;  // P_t: 64 columns of packed bf16
             const uint32_t acc0 = tp ? 1u : 0u;
-            for (int c = 0; c < nch; ++c) {
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
               uint32_t sa;
               if (!ok || !take(sa)) { ok = false; break; }
-              const uint64_t vd = sdesc_sw128(sa, QBOX, 1024);
+              const uint64_t vd = sdesc_sw128(sa, VBOX, 1024);
 #pragma unroll
-              for (int kk = 0; kk < 8; ++kk)
-                umma_bf16_ts(o_tm + c * chw, pa + 8 * kk, vd + ((kk * 2048) >> 4), id_pv,
-                             kk ? 1u : acc0);
+              for (int kk = 0; kk < 4; ++kk)
+                umma_bf16_ts(o_tm, pa + 32 * s + 8 * kk, vd + ((kk * 2048) >> 4), id_pv,
+                             (s | kk) ? 1u : acc0);
               give();
             }
           }
@@ -452,19 +445,16 @@ chunk_out_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ C
         if (!mbar_wait(qt_full, k & 1, 207)) { ok = false; break; }
         tc_fence_after();
         if (x.has_r) {
-          const int rsteps = rrows / 16;  // 16 rows of d_k per MMA
-          for (int dh = 0; dh < p.dk / rrows && ok; ++dh) {
-            for (int c = 0; c < nch; ++c) {
-              uint32_t sa;
-              if (!ok || !take(sa)) { ok = false; break; }
-              const uint64_t rd = sdesc_sw128(sa, rrows * 128, 1024);
-              for (int kk = 0; kk < rsteps; ++kk) {
-                const int row = dh * rrows + 16 * kk;  // d_k row of this step
-                umma_bf16_ss(o_tm + c * chw, qd + ((((row >> 6) * QBOX) + (row & 63) * 2) >> 4),
-                             rd + ((kk * 2048) >> 4), id_pv, 1u);
-              }
-              give();
-            }
+#pragma unroll
+          for (int s = 0; s < KQ; ++s) {
+            uint32_t sa;
+            if (!ok || !take(sa)) { ok = false; break; }
+            const uint64_t rd = sdesc_sw128(sa, VBOX, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_bf16_ss(o_tm, qd + ((s * QBOX + kk * 32) >> 4), rd + ((kk * 2048) >> 4), id_pv,
+                           1u);
+            give();
           }
         }
         umma_commit(o_full);
@@ -785,11 +775,9 @@ cudaError_t launch_tc_out(const void* q, const void* k, const void* v, const flo
   } else {
     tm_g = tm_o;  // never read
   }
-  if ((e = make_tmap_bf16_3d(&tm_v, v, dv, N, BH, 64, BN)) != cudaSuccess) return e;
+  if ((e = make_tmap_bf16_3d(&tm_v, v, dv, N, BH, 64, 64)) != cudaSuccess) return e;
   if (ws) {
-    if ((e = make_tmap_bf16_3d(&tm_r, ws, dv, dk, BH * p.nc, 64, dk < 128 ? dk : 128)) !=
-        cudaSuccess)
-      return e;
+    if ((e = make_tmap_bf16_3d(&tm_r, ws, dv, dk, BH * p.nc, 64, 64)) != cudaSuccess) return e;
   } else {
     tm_r = tm_v;  // never read
   }

@@ -186,12 +186,23 @@ def test_state_combine_rejects_bad_arguments(lib):
 def test_backward_rejects_bad_arguments(lib):
     need = lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 64, 64, 0)
     assert need > 0 and lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 64, 0, 0) == 0
-    # float32 forward and gradient states plus two [c][c] score blocks per chunk of
-    # c = min(chunk, 128) tokens
-    for chunk, c in ((64, 64), (37, 37), (512, 128)):
+    # CUDA-core backward (float32, and bf16 with chunks the tensor cores do not
+    # tile): float32 forward and gradient states plus two [c][c] score blocks
+    # per chunk of c = min(chunk, 128) tokens
+    for dt, chunk, c in ((0, 64, 64), (0, 37, 37), (0, 512, 128), (1, 64, 64), (1, 37, 37)):
         nc = -(-300 // c)
-        assert lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 96, chunk, 1) == \
+        assert lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 96, chunk, dt) == \
             2 * 4 * 2 * nc * (64 * 96 + c * c)
+    # bf16 with a tensor-core chunk: reversed copies of q, k, v and dO, four
+    # float32 states, then the workspace of the forward calls (the larger of
+    # the two mapped shapes), each region rounded up to 256 bytes
+    al = lambda x: -(-x // 256) * 256
+    for chunk in (128, 512):
+        fws = max(lib.ret_chunkwise_workspace(1, 2, 300, 96, 64, chunk, 1),
+                  lib.ret_chunkwise_workspace(1, 2, 300, 64, 96, chunk, 1))
+        want = (2 * al(2 * 300 * 64 * 2) + 2 * al(2 * 300 * 96 * 2) + 4 * al(2 * 64 * 96 * 4)
+                + al(fws))
+        assert lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 96, chunk, 1) == want
 
     def call(q=A, dO=A, gq=A, ds=A, si=None, dso=None, ws=A, wsb=None, N=300, chunk=64, dt=0):
         wsb = need if wsb is None else wsb

@@ -120,6 +120,34 @@ def test_chunkwise_parity(torch_cuda, ret, case):
     assert _rel(s, s_ref) <= STATE_TOL
 
 
+# bf16 shapes outside the tensor-core tiling (chunk not in {128, 256, 512}, or
+# d_k / d_v not a power of two in [64, 256] / [64, 512]) run the float32
+# CUDA-core kernels on the bf16 inputs; their only rounding is the bf16
+# output, so they are held to a tolerance well inside the bf16 one.
+OFF_TC_CASES = [
+    # B, H, N, dk, dv, chunk, gn_eps, state_in
+    (1, 3, 300, 256, 512, 64, 1e-5, True),    # chunk 64
+    (2, 2, 333, 128, 128, 100, None, False),  # chunk not a power of two
+    (1, 2, 200, 32, 64, 128, None, True),     # d_k below the tensor-core tiles
+    (1, 2, 150, 512, 128, 128, None, False),  # d_k above them
+]
+
+
+@pytest.mark.parametrize("case", OFF_TC_CASES, ids=lambda c: "-".join(map(str, c)))
+def test_bf16_outside_tensor_core_tiling_runs_float32_path(torch_cuda, ret, case):
+    torch = torch_cuda
+    B, H, N, dk, dv, chunk, gn, with_s0 = case
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=1200 + N, with_state=with_s0)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    s0 = _dev(inp["state"]) if with_s0 else None
+    o, s = ret.chunkwise(q, k, v, g, chunk, state_in=s0, return_state=True, gn_eps=gn)
+    torch.cuda.synchronize()
+    o_ref, s_ref = _ref_chunkwise(inp, chunk, gn, with_s0)
+    assert _rel(o, o_ref) <= 5e-3            # the bf16 rounding of o alone
+    assert _rel(s, s_ref) <= STATE_TOL
+
+
 def test_chunkwise_without_state_out_and_in_place(torch_cuda, ret):
     torch = torch_cuda
     B, H, N, dk, dv, C = 1, 2, 520, 128, 128, 128
@@ -424,6 +452,32 @@ def test_chunkwise_backward_parity(torch_cuda, ret, case):
     assert _rel(gk, rk) <= tol
     assert _rel(gv, rv) <= tol
     assert _rel(gs, rs) <= (1e-5 if dt == "f32" else 1e-4)
+
+
+def test_chunkwise_backward_bf16_special_decays(torch_cuda, ret):
+    """The bf16 backward runs as three forward calls; the final-state gradient
+    enters two of them divided by gamma, and for gamma = 0 a separate pass
+    adds it at the last token.  Decays 0, 0.5, 0.9 and 1, with incoming and
+    final-state gradients, on a chunk the tensor cores tile."""
+    torch = torch_cuda
+    B, H, N, dk, dv, chunk = 1, 4, 300, 128, 128, 128
+    gam = [0.0, 0.5, 0.9, 1.0]
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=211, with_state=True, gammas=gam)
+    rng = np.random.default_rng(212)
+    d_o = wl.from_values(rng.standard_normal((B, H, N, dv)) * 0.1, "bf16")
+    d_s = rng.standard_normal((B, H, dk, dv)).astype(np.float32)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    gq, gk, gv, gs = ret.chunkwise_backward(q, k, v, g, chunk, _dev(d_o),
+                                            state_in=_dev(inp["state"]),
+                                            d_state_out=torch.from_numpy(d_s).cuda())
+    torch.cuda.synchronize()
+    rq, rk, rv, rs = oracle.backward(inp["q"].exact, inp["k"].exact, inp["v"].exact,
+                                     inp["gammas"], d_o.exact, inp["state"].exact, d_s)
+    assert _rel(gq, rq) <= TOL["bf16"]
+    assert _rel(gk, rk) <= TOL["bf16"]
+    assert _rel(gv, rv) <= TOL["bf16"]
+    assert _rel(gs, rs) <= 1e-4
 
 
 # --- the largest supported sizes and many (batch, head) pairs -------------------
