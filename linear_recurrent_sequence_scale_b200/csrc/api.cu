@@ -251,9 +251,47 @@ int ret_chunkwise(const void* q, const void* k, const void* v, const float* gamm
                              dv, dtype, gn_eps, workspace, workspace_bytes, stream);
 }
 
+}  // extern "C"
+
+namespace {
+
+// The bf16 backward as three forward calls (backward_tc.cu): reversed copies
+// of q, k, v and dO, the prepared states, then the forward calls' workspace.
+struct BwdTcLayout {
+  size_t qr, kr, vr, dor, sin_t, dso_t, dso, g0, fws, fws_bytes, total;
+};
+
+bool bwd_tc(int dtype, int chunk) { return dtype == RET_BF16 && tc_chunk(chunk); }
+
+BwdTcLayout bwd_tc_layout(int B, int H, int N, int dk, int dv, int chunk) {
+  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  const size_t BH = (size_t)B * H;
+  const size_t rk = al(BH * N * dk * 2), rv = al(BH * N * dv * 2), st = al(BH * dk * dv * 4);
+  BwdTcLayout L;
+  L.qr = 0;
+  L.kr = L.qr + rk;
+  L.vr = L.kr + rk;
+  L.dor = L.vr + rv;
+  L.sin_t = L.dor + rv;
+  L.dso_t = L.sin_t + st;
+  L.dso = L.dso_t + st;
+  L.g0 = L.dso + st;
+  L.fws = L.g0 + st;
+  const size_t a = ret_chunkwise_workspace(B, H, N, dv, dk, chunk, RET_BF16);  // dq, dk calls
+  const size_t b = ret_chunkwise_workspace(B, H, N, dk, dv, chunk, RET_BF16);  // the dv call
+  L.fws_bytes = al(a > b ? a : b);
+  L.total = L.fws + L.fws_bytes;
+  return L;
+}
+
+}  // namespace
+
+extern "C" {
+
 size_t ret_chunkwise_backward_workspace(int B, int H, int N, int dk, int dv, int chunk,
                                         int dtype) {
   if (check_seq_dims(B, H, N, dk, dv, dtype) != RET_OK || chunk < 1 || N == 0) return 0;
+  if (bwd_tc(dtype, chunk)) return bwd_tc_layout(B, H, N, dk, dv, chunk).total;
   return ret::backward_workspace_bytes(B, H, N, dk, dv, chunk);
 }
 
@@ -282,12 +320,62 @@ int ret_chunkwise_backward(const void* q, const void* k, const void* v, const fl
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(d_o) || !aligned16(dq) ||
       !aligned16(dk_) || !aligned16(dv_))
     return RET_EINVAL;
-  const size_t need = ret::backward_workspace_bytes(B, H, N, dk, dv, chunk);
+  const size_t need = ret_chunkwise_backward_workspace(B, H, N, dk, dv, chunk, dtype);
   if (!workspace || workspace_bytes < need) return RET_EWORKSPACE;
   if (!aligned16(workspace)) return RET_EINVAL;
-  return cuda_status(ret::launch_chunkwise_backward(q, k, v, gammas, chunk, state_in, d_o,
-                                                    d_state_out, dq, dk_, dv_, d_state_in, B, H,
-                                                    N, dk, dv, dtype, workspace, st));
+  if (!bwd_tc(dtype, chunk))
+    return cuda_status(ret::launch_chunkwise_backward(q, k, v, gammas, chunk, state_in, d_o,
+                                                      d_state_out, dq, dk_, dv_, d_state_in, B,
+                                                      H, N, dk, dv, dtype, workspace, st));
+  // bf16: each gradient is the forward chunkwise form of permuted inputs
+  // (backward_tc.cu states the identities), run by the forward's kernels.
+  const BwdTcLayout L = bwd_tc_layout(B, H, N, dk, dv, chunk);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  void *qr = w + L.qr, *kr = w + L.kr, *vr = w + L.vr, *dor = w + L.dor;
+  float* sin_t = reinterpret_cast<float*>(w + L.sin_t);
+  float* dso_t = reinterpret_cast<float*>(w + L.dso_t);
+  float* dso = reinterpret_cast<float*>(w + L.dso);
+  float* g0 = reinterpret_cast<float*>(w + L.g0);
+  void* fws = w + L.fws;
+  const int BH = B * H;
+  cudaError_t e;
+#define RET_TRY(call)                            \
+  do {                                           \
+    if ((e = (call)) != cudaSuccess) return cuda_status(e); \
+  } while (0)
+#define RET_TRY_STATUS(call)                     \
+  do {                                           \
+    const int s2 = (call);                       \
+    if (s2 != RET_OK) return s2;                 \
+  } while (0)
+  RET_TRY(ret::launch_reverse_rows(q, qr, BH, N, dk, st));
+  RET_TRY(ret::launch_reverse_rows(k, kr, BH, N, dk, st));
+  RET_TRY(ret::launch_reverse_rows(v, vr, BH, N, dv, st));
+  RET_TRY(ret::launch_reverse_rows(d_o, dor, BH, N, dv, st));
+  if (state_in) RET_TRY(ret::launch_prep_state(state_in, sin_t, gammas, BH, H, dk, dv, 1, 0, 0, st));
+  if (d_state_out) {
+    RET_TRY(ret::launch_prep_state(d_state_out, dso_t, gammas, BH, H, dk, dv, 1, 1, 0, st));
+    RET_TRY(ret::launch_prep_state(d_state_out, dso, gammas, BH, H, dk, dv, 0, 1, 0, st));
+  }
+  // dq = forward(dO, V, K; S_in^T)
+  RET_TRY_STATUS(ret_chunkwise(d_o, v, k, gammas, chunk, state_in ? sin_t : nullptr, nullptr, dq,
+                               B, H, N, dv, dk, RET_BF16, -1.f, fws, L.fws_bytes, stream));
+  // dk, reversed = forward(V', dO', Q'; dS_out^T / gamma)
+  RET_TRY_STATUS(ret_chunkwise(vr, dor, qr, gammas, chunk, d_state_out ? dso_t : nullptr, nullptr,
+                               dk_, B, H, N, dv, dk, RET_BF16, -1.f, fws, L.fws_bytes, stream));
+  // dv, reversed = forward(K', Q', dO'; dS_out / gamma), final state G_0
+  RET_TRY_STATUS(ret_chunkwise(kr, qr, dor, gammas, chunk, d_state_out ? dso : nullptr,
+                               d_state_in ? g0 : nullptr, dv_, B, H, N, dk, dv, RET_BF16, -1.f,
+                               fws, L.fws_bytes, stream));
+  RET_TRY(ret::launch_reverse_rows(dk_, dk_, BH, N, dk, st));
+  RET_TRY(ret::launch_reverse_rows(dv_, dv_, BH, N, dv, st));
+  if (d_state_in) RET_TRY(ret::launch_prep_state(g0, d_state_in, gammas, BH, H, dk, dv, 0, 0, 1, st));
+  if (d_state_out)
+    RET_TRY(ret::launch_gamma_zero_last_token(k, v, d_state_out, gammas, dk_, dv_, BH, H, N, dk,
+                                              dv, st));
+#undef RET_TRY
+#undef RET_TRY_STATUS
+  return RET_OK;
 }
 
 int ret_state_combine(const float* locals, const int* spans, int r, const float* gammas,

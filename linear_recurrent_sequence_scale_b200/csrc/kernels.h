@@ -34,6 +34,16 @@ cudaError_t launch_chunkwise_backward(const void* q, const void* k, const void* 
                                       int N, int dk, int dv, int dtype, void* ws,
                                       cudaStream_t st);
 
+// Data movement for the bf16 backward built from forward calls (backward_tc.cu).
+cudaError_t launch_reverse_rows(const void* src, void* dst, int BH, int N, int d,
+                                cudaStream_t st);
+cudaError_t launch_prep_state(const float* in, float* out, const float* gammas, int BH, int H,
+                              int R, int C, int transpose, int inv_gamma, int by_gamma,
+                              cudaStream_t st);
+cudaError_t launch_gamma_zero_last_token(const void* k, const void* v, const float* ds,
+                                         const float* gammas, void* dk, void* dv, int BH, int H,
+                                         int N, int DK, int DV, cudaStream_t st);
+
 // State entering span r of a sequence split across GPUs (seqpar.cu).
 constexpr int kMaxSpans = 64;
 cudaError_t launch_state_combine(const float* locals, const int* spans, int r,
