@@ -117,21 +117,6 @@ __device__ __forceinline__ int tile_at(const Params& p, int k) {
   return t < p.ntiles ? t : -1;
 }
 
-// Chan et al.: merge (n_b, mean_b, m2_b) into (n_a, mean_a, m2_a).
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, uint32_t src, int x, int y,
-                                             int z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(m)),
-      "r"(src), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_commit() {
-  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read0() {
-  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
 // Named barriers of the epilogue warps (0 is __syncthreads).
 // Barrier 1 also ANDs a flag over the epilogue warps, so that they leave the
 // tile loop together when a wait has failed and never strand each other on a

@@ -26,6 +26,8 @@
 // (one chunk), so the float32 state stays accurate over any sequence length.
 // MH = 2 halves the number of CTAs reading each K tile; MH = 1 gives twice
 // the CTAs for small batches.
+#include <string.h>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -49,11 +51,17 @@ constexpr int LO_OFF = 6 * BOX;        // 2 boxes (V lo, with the hi/lo split on
 template <bool SPLIT> struct Ring {
   static constexpr int STAGES = SPLIT ? 3 : 4;
   static constexpr int STAGE_BYTES = (SPLIT ? 8 : 6) * BOX;
-  static constexpr int BAR_OFF = STAGES * STAGE_BYTES;
 };
-constexpr int SMEM_BYTES = 3 * 8 * BOX + 512 + 1024;
-static_assert(Ring<true>::BAR_OFF + 512 + 1024 <= SMEM_BYTES &&
-              Ring<false>::BAR_OFF + 512 + 1024 <= SMEM_BYTES, "ring fits");
+// After the ring: one 4 KB staging box per state warp (32 state rows x 64
+// columns of bf16, 128-byte swizzle) through which the chunk states leave by
+// TMA, then the mbarriers.
+constexpr int STG_OFF = 3 * 8 * BOX;
+constexpr int STG_BYTES = 32 * 128;
+constexpr int BAR_OFF = STG_OFF + 8 * STG_BYTES;
+constexpr int SMEM_BYTES = BAR_OFF + 512 + 1024;
+static_assert(Ring<true>::STAGES * Ring<true>::STAGE_BYTES <= STG_OFF &&
+              Ring<false>::STAGES * Ring<false>::STAGE_BYTES <= STG_OFF, "ring fits");
+static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per CTA");
 constexpr int XF_WARPS = 8;            // V (.) zeta warps
 #ifndef RET_K2_XG
 #define RET_K2_XG 1
@@ -76,18 +84,18 @@ struct Params {
   __nv_bfloat16* ws;  // [B*H*nc][dk][dv]; slot i = state entering chunk i
   int H, N, chunk, nc, dk, dv, nt, mh;
   int write_ws0;      // store state_in (as bf16) in slot 0
+  int tma_ws;         // chunk states stored by TMA (64-column halves of NT)
 };
 
 template <bool SPLIT, int MH>
 __global__ void __launch_bounds__(THREADS, 1)
 state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-              const Params p) {
+              const __grid_constant__ CUtensorMap tm_ws, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   constexpr int STAGES = Ring<SPLIT>::STAGES;
   constexpr int STAGE_BYTES = Ring<SPLIT>::STAGE_BYTES;
-  constexpr int BAR_OFF = Ring<SPLIT>::BAR_OFF;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
   uint64_t* full = bars;                 // TMA -> transform
   uint64_t* xf = bars + STAGES;          // transform -> MMA
@@ -336,6 +344,11 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(h_free);
+      // the new state from TMEM to memory: bf16 to the workspace (staged per
+      // warp in shared memory and stored by TMA as one [32 rows][64 columns]
+      // box), or float32 to state_out after the last chunk
+      const uint32_t stg = smem_u32(smem + STG_OFF + (warp - EPI_WARP0) * STG_BYTES);
+      const bool by_tma = !last && p.tma_ws;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         if (hh >= p.mh) continue;
@@ -348,6 +361,23 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
           uint32_t v[32];
           tmem_ld32(tmem + rcol + hoff, v);  // warp-wide: every lane loads
           tmem_wait_ld();
+          if (by_tma) {
+            // the previous box's store has read this warp's staging
+            if (x0 == 0) {
+              if (lane == 0) bulk_wait_read0();
+              __syncwarp();
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+              const int c = (x0 / 8 + x) ^ (lane & 7);  // 128-byte swizzle
+              st_shared_v4(stg + lane * 128 + c * 16,
+                           pack_bf16(__uint_as_float(v[8 * x]), __uint_as_float(v[8 * x + 1])),
+                           pack_bf16(__uint_as_float(v[8 * x + 2]), __uint_as_float(v[8 * x + 3])),
+                           pack_bf16(__uint_as_float(v[8 * x + 4]), __uint_as_float(v[8 * x + 5])),
+                           pack_bf16(__uint_as_float(v[8 * x + 6]), __uint_as_float(v[8 * x + 7])));
+            }
+            continue;
+          }
           if (!live) continue;
           if (!last) {
             uint4* dst = reinterpret_cast<uint4*>(
@@ -368,8 +398,20 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                                    __uint_as_float(v[4 * x + 2]), __uint_as_float(v[4 * x + 3]));
           }
         }
+        if (by_tma) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          const int rb = r0 + 128 * hh + 32 * q;  // first row of the box
+          if (lane == 0 && rb < p.dk) {
+            tma_store_3d(&tm_ws, stg, cb, rb, bh * p.nc + ci + 1);
+            bulk_commit();
+          }
+        }
       }
     }
+    // the staging must have been read before the CTA's shared memory goes
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -394,6 +436,16 @@ cudaError_t launch_tc_state(const void* k, const void* v, const float* gammas, i
   if (e != cudaSuccess) return e;
   e = make_tmap_bf16_3d(&tm_v, v, dv, N, BH, 64, T);
   if (e != cudaSuccess) return e;
+  // chunk-state boxes of [32 rows][64 columns] (state columns per warp: 64
+  // unless d_v = 64, which keeps plain stores)
+  CUtensorMap tm_ws;
+  memset(&tm_ws, 0, sizeof(tm_ws));
+  const int nc = cdiv(N, chunk);
+  const int tma_ws = ws != nullptr && nc > 1 && dv >= NT ? 1 : 0;
+  if (tma_ws) {
+    e = make_tmap_bf16_3d(&tm_ws, ws, dv, dk, BH * nc, 64, 32);
+    if (e != cudaSuccess) return e;
+  }
   Params p;
   p.gammas = gammas;
   p.state_in = state_in;
@@ -407,6 +459,7 @@ cudaError_t launch_tc_state(const void* k, const void* v, const float* gammas, i
   p.dv = dv;
   p.nt = dv < NT ? dv : NT;
   p.write_ws0 = write_ws0;
+  p.tma_ws = tma_ws;
   // Both d_k halves in one CTA (K read by half as many CTAs) when that still
   // gives at least one CTA per SM; otherwise one half per CTA.
   int dev = 0, nsm = 148;
@@ -419,7 +472,7 @@ cudaError_t launch_tc_state(const void* k, const void* v, const float* gammas, i
     cudaError_t e2 = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           SMEM_BYTES);
     if (e2 != cudaSuccess) return e2;
-    fn<<<grid, THREADS, SMEM_BYTES, st>>>(tm_k, tm_v, p);
+    fn<<<grid, THREADS, SMEM_BYTES, st>>>(tm_k, tm_v, tm_ws, p);
     return cudaPeekAtLastError();
   };
   if (state_out) return p.mh == 2 ? go(state_scan_tc<true, 2>) : go(state_scan_tc<true, 1>);
