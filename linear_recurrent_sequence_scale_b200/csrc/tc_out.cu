@@ -148,6 +148,20 @@ __device__ __forceinline__ void chan_merge(float& n_a, float& mean_a, float& m2_
   n_a = n;
 }
 
+// swish(x) = x sigmoid(x) with sigmoid(x) = (1 + tanh(x / 2)) / 2 and the
+// hardware tanh approximation: one special-function op per element instead
+// of an exponential and a division.  The epilogue runs it on every output
+// element, and the special-function unit is what bounds the gated tile
+// (output phase on the 8k workload: 2.21 ms with exp and an IEEE division,
+// 1.49 ms with fast exp and reciprocal, 1.34 ms with tanh; 1.29 ms ungated).
+// The absolute error of sigmoid stays near 2^-12, far below the bf16
+// rounding of the gated output at the scale of the tile.
+__device__ __forceinline__ float swish_tanh(float x) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+  return x * fmaf(0.5f, t, 0.5f);
+}
+
 // y <- y swish(g) on eight bf16 values (four packed pairs), g read from the
 // staged gate piece at the same place.
 __device__ __forceinline__ void gate_in_place(uint32_t& y0, uint32_t& y1, uint32_t& y2,
@@ -156,8 +170,8 @@ __device__ __forceinline__ void gate_in_place(uint32_t& y0, uint32_t& y1, uint32
   const uint32_t gi[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
   for (int e = 0; e < 4; ++e)
-    *y[e] = pack_bf16(bf16lo_to_f32(*y[e]) * swishf(bf16lo_to_f32(gi[e])),
-                      bf16hi_to_f32(*y[e]) * swishf(bf16hi_to_f32(gi[e])));
+    *y[e] = pack_bf16(bf16lo_to_f32(*y[e]) * swish_tanh(bf16lo_to_f32(gi[e])),
+                      bf16hi_to_f32(*y[e]) * swish_tanh(bf16hi_to_f32(gi[e])));
 }
 
 // Sum of 32 values as a balanced tree: depth 5 instead of a 32-long chain.

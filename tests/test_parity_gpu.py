@@ -355,6 +355,30 @@ def test_gated_output_phase(torch_cuda, ret):
     assert _rel(o, oracle.gated(y_ref, gate.exact)) <= TOL["bf16"]
 
 
+def test_gated_tensor_cores_across_the_gate_range(torch_cuda, ret):
+    """The tensor-core epilogue takes sigmoid through the hardware tanh; gates
+    spread over [-12, 12] (saturated tails on both sides, where 1 + tanh
+    cancels) stay within the bf16 tolerance per 128-row tile, and the
+    elementwise error of the gate factor stays below 2^-8 of |g| + 1."""
+    torch = torch_cuda
+    B, H, N, dk, dv, C = 1, 2, 1024, 256, 512, 512
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=75)
+    gate = wl.from_values(np.random.default_rng(76).uniform(-12.0, 12.0, (B, H, N, dv)), "bf16")
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    o0 = ret.chunkwise(q, k, v, g, C, gn_eps=1e-5)
+    o1 = ret.chunkwise(q, k, v, g, C, gn_eps=1e-5, gate=_dev(gate))
+    torch.cuda.synchronize()
+    y_ref, _ = _ref_chunkwise(inp, C, 1e-5, False)
+    assert _rel(o1, oracle.gated(y_ref, gate.exact)) <= TOL["bf16"]
+    # the gate factor itself, against the ungated output of the same kernel
+    y = wl.from_torch(o0).astype(np.float64)
+    want = oracle.gated(y, gate.exact)
+    got = wl.from_torch(o1).astype(np.float64)
+    err = np.abs(got - want) - 2.0 ** -8 * np.abs(want)   # beyond the bf16 rounding
+    assert np.max(err / (np.abs(y) * (np.abs(gate.exact) + 1.0) + 1e-30)) <= 2.0 ** -8
+
+
 def test_gate_none_is_the_ungated_call(torch_cuda, ret):
     """gate=None runs the ungated entry point; a gate of +40 (swish(40) = 40
     in bf16 arithmetic) scales the ungated result by 40."""
