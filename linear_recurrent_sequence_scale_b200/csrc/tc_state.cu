@@ -97,10 +97,11 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
   constexpr int STAGES = Ring<SPLIT>::STAGES;
   constexpr int STAGE_BYTES = Ring<SPLIT>::STAGE_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
-  uint64_t* full = bars;                 // TMA -> transform
+  uint64_t* full = bars;                 // TMA (V) -> transform
   uint64_t* xf = bars + STAGES;          // transform -> MMA
   uint64_t* empty = bars + 2 * STAGES;   // MMA -> TMA
-  uint64_t* h_full = bars + 3 * STAGES;  // MMA -> epilogue
+  uint64_t* full_k = bars + 3 * STAGES;  // TMA (K) -> MMA
+  uint64_t* h_full = bars + 4 * STAGES;  // MMA -> epilogue
   uint64_t* h_free = h_full + 1;         // epilogue -> MMA
   uint64_t* drain = h_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(h_full + 3);
@@ -123,6 +124,7 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
+      mbar_init(&full_k[s], 1);
       mbar_init(&xf[s], XF_WARPS / XG);
       mbar_init(&empty[s], 1);
     }
@@ -156,16 +158,21 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
           const int slot = g % STAGES;
           if (!mbar_wait(&empty[slot], ((g / STAGES) & 1) ^ 1, 101)) { ok = false; break; }
           uint8_t* st = smem + slot * STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[slot], (kboxes + vboxes) * BOX);
-          for (int b = 0; b < kboxes; ++b)
-            tma_load_3d(st + K_OFF + b * BOX, &tm_k, &full[slot], r0 + b * 64, cs + j0, bh);
+          // V first, on its own barrier: the transform starts on it while K
+          // (needed only by the MMA) is still landing
+          mbar_arrive_expect_tx(&full[slot], vboxes * BOX);
+          mbar_arrive_expect_tx(&full_k[slot], kboxes * BOX);
           for (int b = 0; b < vboxes; ++b)
             tma_load_3d(st + V_OFF + b * BOX, &tm_v, &full[slot], c0 + b * 64, cs + j0, bh);
+          for (int b = 0; b < kboxes; ++b)
+            tma_load_3d(st + K_OFF + b * BOX, &tm_k, &full_k[slot], r0 + b * 64, cs + j0, bh);
         }
       }
       // no copy may still be landing when the CTA exits
-      for (int gg = max(0, g - STAGES); gg < g; ++gg)
+      for (int gg = max(0, g - STAGES); gg < g; ++gg) {
         mbar_wait(&full[gg % STAGES], (gg / STAGES) & 1, 108);
+        mbar_wait(&full_k[gg % STAGES], (gg / STAGES) & 1, 108);
+      }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -188,7 +195,8 @@ state_scan_tc(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         bool first = true;
         for (int j0 = 0; j0 < L; j0 += T, ++g) {
           const int slot = g % STAGES;
-          if (!mbar_wait(&xf[slot], (g / STAGES) & 1, 103)) { ok = false; break; }
+          if (!mbar_wait(&xf[slot], (g / STAGES) & 1, 103) ||
+              !mbar_wait(&full_k[slot], (g / STAGES) & 1, 110)) { ok = false; break; }
           tc_fence_after();
           const uint64_t so = static_cast<uint64_t>((slot * STAGE_BYTES) >> 4);
 #pragma unroll
