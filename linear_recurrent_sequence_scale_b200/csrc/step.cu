@@ -35,7 +35,21 @@ namespace ret {
 constexpr int STEP_COLS = 128;
 constexpr int STEP_THREADS = 256;
 constexpr int STEP_RG = STEP_THREADS / (STEP_COLS / 4);  // 8 row groups (= warps)
-constexpr int STEP_UNROLL = 8;
+// Residency.  The grid is d_v/128 x B x H CTAs of equal work (512 for the
+// 6.7B-class layer at batch 8), all streaming the state at once; what decides
+// the time is how evenly they fill the SMs.  Three CTAs per SM (the
+// register count the compiler picks by default) run 444 of 512 in a first
+// wave and leave a 68-CTA tail: 28.5 us per step.  Without GroupNorm, two
+// per SM with eight row loads in flight per warp take 25.0 us (two waves of
+// 296 and 216 CTAs, each with ~9 MB of loads in flight); the residency is
+// pinned by the shared-memory request (STEP_SMEM_FLOOR), not left to the
+// register count.  With GroupNorm (4-CTA clusters) four per SM with four
+// row loads in flight, a single wave, measured best (27.3 against 29.3 us).
+template <bool GN> struct StepCfg {
+  static constexpr int UNROLL = GN ? 4 : 8;
+  static constexpr int MIN_BLOCKS = GN ? 4 : 1;
+};
+constexpr size_t STEP_SMEM_FLOOR = 80 * 1024;  // > 1/3 of an SM's shared memory
 
 __device__ __forceinline__ float block_sum_256(float x, float* scratch /* >= 8 floats */) {
 #pragma unroll
@@ -51,7 +65,7 @@ __device__ __forceinline__ float block_sum_256(float x, float* scratch /* >= 8 f
 }
 
 template <typename T, bool GN, bool ROT>
-__global__ void __launch_bounds__(STEP_THREADS)
+__global__ void __launch_bounds__(STEP_THREADS, StepCfg<GN>::MIN_BLOCKS)
 step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
             const float* __restrict__ gammas, float* __restrict__ state,
             const T* __restrict__ gate, T* __restrict__ o, int H, int dk, int dv, float eps,
@@ -101,6 +115,7 @@ step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
   if (cval) vv = Elem<T>::ld4(v + (size_t)bh * dv + c);
   __syncthreads();
 
+  constexpr int STEP_UNROLL = StepCfg<GN>::UNROLL;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float* S = state + (size_t)bh * dk * dv + c;
   for (int r0 = rg; r0 < dk; r0 += STEP_RG * STEP_UNROLL) {
@@ -178,7 +193,9 @@ static cudaError_t launch_step_t(const void* q, const void* k, const void* v, co
                                  cudaStream_t st) {
   const int nct = cdiv(dv, STEP_COLS);
   dim3 grid(nct, B * H);
-  const size_t smem = sizeof(float) * (2 * dk + STEP_RG * STEP_COLS);
+  const size_t need = sizeof(float) * (2 * dk + STEP_RG * STEP_COLS);
+  // without GroupNorm at most two CTAs per SM (see StepCfg)
+  const size_t smem = eps < 0.f && need < STEP_SMEM_FLOOR ? STEP_SMEM_FLOOR : need;
   const T* qq = static_cast<const T*>(q);
   const T* kk = static_cast<const T*>(k);
   const T* vv = static_cast<const T*>(v);
