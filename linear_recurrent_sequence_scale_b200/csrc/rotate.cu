@@ -14,10 +14,13 @@
 // depends on (n, c) only, so a thread takes the cos / sin of its V channel
 // pairs once, in double precision (n theta reaches 1e6 rad and more, where a
 // float32 product would lose the phase), and applies them to the same
-// (n, pairs) of up to kRowsPerThread (batch, head) rows.  Rows are handled
-// four at a time, all four loaded before any is stored, which keeps several
-// loads in flight per thread and is safe in place (y == x): every element is
-// read and written by the one thread that owns it.
+// (n, pairs) of up to kRowsPerThread (batch, head) rows, one row at a time
+// (kGroup rows would be loaded before any is stored).  More rows in flight
+// per thread measured slower: each is a different (batch, head) block 4 MB
+// away, so a warp's loads then spread over kGroup DRAM pages at once (8k
+// workload, q and k in place: 4 rows 4804 GB/s, 2 rows 5533, 1 row 5748; 32
+// rows per thread instead of 16: 5789).  In place (y == x) is safe: every
+// element is read and written by the one thread that owns it.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -25,8 +28,8 @@ namespace ret {
 namespace rot {
 
 constexpr int kThreads = 256;
-constexpr int kRowsPerThread = 16;  // (batch, head) rows sharing one set of angles
-constexpr int kGroup = 4;           // rows loaded together
+constexpr int kRowsPerThread = 32;  // (batch, head) rows sharing one set of angles
+constexpr int kGroup = 1;           // rows loaded together
 
 template <typename T, int V>
 struct Pairs {

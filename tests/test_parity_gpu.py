@@ -99,6 +99,8 @@ CHUNK_CASES = [
     ("bf16", 1, 4, 333, 64, 64, 128, None, True),
     ("bf16", 2, 2, 640, 128, 128, 256, 1e-5, False),
     ("bf16", 1, 2, 1100, 128, 512, 256, None, True),
+    ("bf16", 2, 3, 600, 64, 256, 128, None, True),     # d_k 64: state boxes past d_k skipped
+    ("bf16", 10, 4, 600, 256, 512, 256, 1e-5, False),  # 160 column tiles: both d_k halves per CTA
     ("f32", 1, 3, 301, 128, 64, 37, None, True),
     ("f32", 2, 2, 200, 64, 96, 64, 1e-5, False),
     ("f32", 1, 2, 130, 32, 40, 1, None, True),
@@ -118,6 +120,24 @@ def test_chunkwise_parity(torch_cuda, ret, case):
     o_ref, s_ref = _ref_chunkwise(inp, chunk, gn, with_s0)
     assert _rel(o, o_ref) <= TOL[dt]
     assert _rel(s, s_ref) <= STATE_TOL
+
+
+@pytest.mark.parametrize("case", [c for c in CHUNK_CASES if c[0] == "bf16"],
+                         ids=lambda c: "-".join(map(str, c)))
+def test_chunkwise_parity_without_final_state(torch_cuda, ret, case):
+    """The same calls without the final state: the state scan then runs its
+    other variant (no hi/lo split, a deeper ring), whose bf16 chunk states
+    the output kernel reads."""
+    torch = torch_cuda
+    dt, B, H, N, dk, dv, chunk, gn, with_s0 = case
+    inp = wl.make_inputs(B, H, N, dk, dv, dt, seed=200 + N, with_state=with_s0)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    s0 = _dev(inp["state"]) if with_s0 else None
+    o = ret.chunkwise(q, k, v, g, chunk, state_in=s0, gn_eps=gn)
+    torch.cuda.synchronize()
+    o_ref, _ = _ref_chunkwise(inp, chunk, gn, with_s0)
+    assert _rel(o, o_ref) <= TOL[dt]
 
 
 # bf16 shapes outside the tensor-core tiling (chunk not in {128, 256, 512}, or
