@@ -468,13 +468,23 @@ cudaError_t launch_tc_state(const void* k, const void* v, const float* gammas, i
   p.nt = dv < NT ? dv : NT;
   p.write_ws0 = write_ws0;
   p.tma_ws = tma_ws;
-  // Both d_k halves in one CTA (K read by half as many CTAs) when that still
-  // gives at least one CTA per SM; otherwise one half per CTA.
+  // Both d_k halves in one CTA (K read by half as many CTAs, 1.5x the bytes
+  // per stage) or one half per CTA (twice the CTAs): a CTA walks its whole
+  // sequence, one CTA per SM, so the time goes as the number of rounds of
+  // CTAs over the SMs times the bytes each stage loads; take the smaller.
+  // (8k layer at batch 8: 4 rounds x 6 boxes against 7 x 4, both halves;
+  // 1.3B layer: 1 x 6 against 2 x 4, both halves; 64k at batch 1: 1 x 4
+  // against 1 x 6, one half.)
   int dev = 0, nsm = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   const int halves = cdiv(dk, 128);
-  p.mh = (halves == 2 && BH * (uint64_t)(dv / p.nt) >= (uint64_t)nsm) ? 2 : 1;
+  const uint64_t tiles = BH * (uint64_t)(dv / p.nt);
+  auto cost = [&](int mh) {
+    const uint64_t ctas = tiles * (uint64_t)(halves / mh);
+    return ((ctas + nsm - 1) / nsm) * (uint64_t)(2 * mh + p.nt / 64);
+  };
+  p.mh = (halves == 2 && cost(2) < cost(1)) ? 2 : 1;
   dim3 grid(dv / p.nt, halves / p.mh, (unsigned)BH);
   auto go = [&](auto fn) -> cudaError_t {
     cudaError_t e2 = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
