@@ -9,7 +9,9 @@
 //
 // One CTA owns one (batch, head), MH (1 or 2) 128-row halves of d_k and NT
 // (<= 128) state columns, and walks the chunks in order:
-//   warp 0      TMA: K tile [T tokens][128 MH d_k] and V tile [T][NT] per stage
+//   warp 0      TMA: V tile [T tokens][NT] and K tile [T][128 MH d_k] per
+//               stage, each on its own mbarrier (V first: the transform
+//               needs only V, the MMA both)
 //   warps 2-9   V (.) zeta; when the final state is requested it is split
 //               into bf16 hi + lo parts (16 mantissa bits of the product
 //               reach the tensor core instead of 8), hi written in place of V
@@ -20,12 +22,16 @@
 //               chunk end they read H_i (then hand the accumulator back to the
 //               MMA warp), form gamma^L R + H_i with IEEE float32 FMAs, write
 //               R back, and store it as bf16 to the workspace (the state
-//               entering the next chunk, read by the output kernel) or, after
-//               the last chunk, as the float32 final state.
+//               entering the next chunk, read by the output kernel; staged
+//               per warp in shared memory and written by TMA, since 16-byte
+//               stores of every thread's own row cost the transform its
+//               shared-memory bandwidth) or, after the last chunk, as the
+//               float32 final state.
 // Accumulating each chunk afresh keeps the tensor core's running sums short
 // (one chunk), so the float32 state stays accurate over any sequence length.
 // MH = 2 halves the number of CTAs reading each K tile; MH = 1 gives twice
-// the CTAs for small batches.
+// the CTAs for small batches (the launcher picks by rounds of CTAs times
+// bytes per stage).
 #include <string.h>
 
 #include "common.cuh"
