@@ -38,7 +38,7 @@
  *    kernel while it runs surface on the stream like any CUDA error.
  *  - Accumulation is float32.  With RET_BF16 inputs the products run on the
  *    tensor cores with bf16 operands where the shapes fit their tiles (the
- *    rules under each call); other bf16 shapes (chunk 64, dk 32, dk 512 ...)
+ *    rules under each call); other bf16 shapes (chunk 100, dk 32, dk 512 ...)
  *    run the float32 CUDA-core kernels on the same inputs, whose only bf16
  *    rounding is that of o.  Either way o is rounded to the input type.
  */
@@ -99,8 +99,13 @@ RET_API size_t ret_chunkwise_workspace(int B, int H, int N, int dk, int dv, int 
  * The final state is accurate to float32 accumulation (the bf16 path splits
  * the decayed V operand into two bf16 halves when state_out is requested).
  * Supported: chunk >= 1 with either type.  RET_BF16 runs on the tensor cores
- * for chunk in {128, 256, 512} under the dk/dv rules of ret_parallel, and on
- * the float32 CUDA-core kernels otherwise (chunk 64, for instance).
+ * for chunk in {64, 128, 256, 512} under the dk/dv rules of ret_parallel, and
+ * on the float32 CUDA-core kernels otherwise (chunk 100, for instance).  The
+ * tensor-core kernels tile 128 query rows, so chunk 64 runs as 128-token
+ * chunks: every chunk length gives the same o and final state in exact
+ * arithmetic, and only the places where the bf16 copies of the chunk state
+ * are rounded move (every 128 tokens instead of 64).  The workspace size and
+ * the chunk states in it follow that 128-token chunking.
  */
 RET_API int ret_chunkwise(const void* q, const void* k, const void* v, const float* gammas, int chunk,
                   const float* state_in, float* state_out, void* o,
@@ -117,7 +122,8 @@ RET_API int ret_chunkwise(const void* q, const void* k, const void* v, const flo
  *
  * ret_chunkwise_states: from k, v and the decays, writes into `workspace` the
  *   state entering every chunk (slot i = R_{i-1}; slot 0 = state_in when
- *   given) and, when state_out is not NULL, the final float32 state.  It
+ *   given; on the tensor cores chunks of at least 128 tokens, see above) and,
+ *   when state_out is not NULL, the final float32 state.  It
  *   launches nothing when there is a single chunk and no state enters or
  *   leaves.  Arguments as for ret_chunkwise.
  * ret_chunkwise_output: from q, k, v, the decays and the workspace that
@@ -262,13 +268,20 @@ RET_API int ret_state_combine(const float* locals, const int* spans, int r, cons
  *   d_state_in   : [B][H][dk][dv] float32, the gradient of state_in (or NULL)
  *   state_in     : the forward call's initial state, or NULL (zero)
  *   d_state_out  : [B][H][dk][dv] float32, or NULL (zero)
- *   workspace    : at least ret_chunkwise_backward_workspace() bytes; holds
- *                  the forward and the gradient chunk states and the masked
- *                  in-chunk scores, all float32, for chunks of
- *                  min(chunk, 128) tokens (the gradients do not depend on
- *                  the chunk length).
- * Runs on the CUDA cores in float32 for either dtype and any chunk >= 1,
- * dk, dv in [8, 512].  Errors as for ret_chunkwise.
+ *   workspace    : at least ret_chunkwise_backward_workspace() bytes.
+ * RET_BF16 with chunk in {64, 128, 256, 512}: each gradient of the
+ * recurrence is itself a retention operation, so the call runs three forward
+ * chunkwise calls (dq = forward(dO, V, K) with the incoming state S_in^T;
+ * in reversed time dk = forward(V, dO, Q) and dv = forward(K, Q, dO), whose
+ * final state gives d_state_in), on the tensor cores wherever their mapped
+ * shapes fit the tiles of ret_chunkwise; the workspace then holds reversed
+ * copies of q, k, v and dO, four float32 states and the forward calls'
+ * workspace.  Otherwise (float32, or other chunks) it runs the chain rule on
+ * the CUDA cores in float32, its workspace holding the forward and gradient
+ * chunk states and the masked in-chunk scores for chunks of min(chunk, 128)
+ * tokens (the gradients do not depend on the chunk length).
+ * Supported: any chunk >= 1, dk, dv in [8, 512].  Errors as for
+ * ret_chunkwise.
  */
 RET_API size_t ret_chunkwise_backward_workspace(int B, int H, int N, int dk, int dv, int chunk,
                                         int dtype);

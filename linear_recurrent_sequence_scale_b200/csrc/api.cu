@@ -39,7 +39,13 @@ bool pow2_in(int x, int lo, int hi) { return x >= lo && x <= hi && (x & (x - 1))
 
 // Shapes the tensor-core kernels handle (bf16 only).
 bool tc_dims(int dk, int dv) { return pow2_in(dk, 64, 256) && pow2_in(dv, 64, 512); }
-bool tc_chunk(int chunk) { return pow2_in(chunk, 128, 512); }
+bool tc_chunk(int chunk) { return pow2_in(chunk, 64, 512); }
+// The chunk length the tensor-core kernels work in.  Their row tiles hold 128
+// query rows, so a 64-token chunk runs as 128-token chunks: every chunk
+// length gives the same output and final state in exact arithmetic (the
+// chunkwise form regroups one sum), and this moves only where the bf16
+// copies of the carried state are rounded, every 128 tokens instead of 64.
+int tc_tile(int chunk) { return chunk < 128 ? 128 : chunk; }
 
 size_t tc_workspace_bytes(int B, int H, int N, int dk, int dv, int chunk) {
   const size_t nc = (size_t)((N + chunk - 1) / chunk);
@@ -108,7 +114,7 @@ size_t ret_chunkwise_workspace(int B, int H, int N, int dk, int dv, int chunk, i
   if (check_seq_dims(B, H, N, dk, dv, dtype) != RET_OK || chunk < 1) return 0;
   if (N == 0) return 0;
   if (dtype == RET_BF16 && tc_dims(dk, dv) && tc_chunk(chunk))
-    return tc_workspace_bytes(B, H, N, dk, dv, chunk);
+    return tc_workspace_bytes(B, H, N, dk, dv, tc_tile(chunk));
   return ret::simt_workspace_bytes(B, H, N, dk, dv, chunk);
 }
 
@@ -132,8 +138,9 @@ int check_chunkwise(int B, int H, int N, int dk, int dv, int dtype, int chunk,
   if (need > 0 && (!workspace || workspace_bytes < need)) return RET_EWORKSPACE;
   if (workspace && !aligned16(workspace)) return RET_EINVAL;
   if (tc_config(dtype, dk, dv, chunk)) {
-    const int nc = (N + chunk - 1) / chunk;
-    if ((int64_t)nc * (chunk / 128) > 65535) return RET_EUNSUPPORTED;
+    const int c = tc_tile(chunk);
+    const int nc = (N + c - 1) / c;
+    if ((int64_t)nc * (c / 128) > 65535) return RET_EUNSUPPORTED;
   }
   return RET_OK;
 }
@@ -164,9 +171,10 @@ int ret_chunkwise_states(const void* k, const void* v, const float* gammas, int 
   if (tc_config(dtype, dk, dv, chunk)) {
     // Needed whenever a state enters, crosses a chunk boundary or is
     // returned; the incoming state is also stored in workspace slot 0.
-    const int nc = (N + chunk - 1) / chunk;
+    const int c = tc_tile(chunk);
+    const int nc = (N + c - 1) / c;
     if (nc == 1 && !state_out && !state_in) return RET_OK;
-    return cuda_status(ret::launch_tc_state(k, v, gammas, chunk, state_in, state_out, workspace,
+    return cuda_status(ret::launch_tc_state(k, v, gammas, c, state_in, state_out, workspace,
                                             state_in != nullptr, B, H, N, dk, dv, st));
   }
   return cuda_status(ret::launch_simt_states(k, v, gammas, chunk, state_in, state_out, B, H, N,
@@ -192,8 +200,9 @@ int chunkwise_output_impl(const void* q, const void* k, const void* v, const flo
   if (gate && !aligned16(gate)) return RET_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tc_config(dtype, dk, dv, chunk))
-    return cuda_status(ret::launch_tc_out(q, k, v, gammas, chunk, workspace, has_state_in != 0,
-                                          gate, o, B, H, N, dk, dv, gn_eps, 0, after_states, st));
+    return cuda_status(ret::launch_tc_out(q, k, v, gammas, tc_tile(chunk), workspace,
+                                          has_state_in != 0, gate, o, B, H, N, dk, dv, gn_eps, 0,
+                                          after_states, st));
   return cuda_status(ret::launch_simt_output(q, k, v, gammas, chunk, gate, o, B, H, N, dk, dv,
                                              dtype, gn_eps, workspace, st));
 }
@@ -238,7 +247,7 @@ int ret_chunkwise_gated(const void* q, const void* k, const void* v, const float
   if (s) return s;
   // the states kernel ran (and may still be draining) unless nothing needed it
   const bool scanned = tc_config(dtype, dk, dv, chunk) &&
-                       ((N + chunk - 1) / chunk > 1 || state_out || state_in);
+                       ((N + tc_tile(chunk) - 1) / tc_tile(chunk) > 1 || state_out || state_in);
   return chunkwise_output_impl(q, k, v, gammas, chunk, state_in != nullptr, gate, o, B, H, N, dk,
                                dv, dtype, gn_eps, workspace, workspace_bytes, stream, scanned);
 }

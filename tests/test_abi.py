@@ -183,13 +183,28 @@ def test_state_combine_rejects_bad_arguments(lib):
     assert f(r=65) == ret.RET_EUNSUPPORTED
 
 
+def test_bf16_chunk_64_takes_the_tensor_core_layout(lib):
+    """bf16 chunk 64 runs on the tensor-core kernels as 128-token chunks: its
+    workspace is the 128-chunk one (2 bytes per state element, one state per
+    128 tokens), while float32 chunk 64, and bf16 shapes the tensor cores do
+    not tile, keep the CUDA-core layout."""
+    for B, H, N, dk, dv in ((1, 2, 300, 64, 64), (2, 3, 1000, 256, 512), (1, 1, 128, 128, 256)):
+        tc128 = lib.ret_chunkwise_workspace(B, H, N, dk, dv, 128, 1)
+        assert tc128 == 2 * B * H * -(-N // 128) * dk * dv
+        assert lib.ret_chunkwise_workspace(B, H, N, dk, dv, 64, 1) == tc128
+        assert lib.ret_chunkwise_workspace(B, H, N, dk, dv, 64, 0) != tc128
+    # d_k 32 is outside the tensor-core tiles: chunk 64 stays on the CUDA cores
+    assert lib.ret_chunkwise_workspace(1, 2, 300, 32, 64, 64, 1) == \
+        lib.ret_chunkwise_workspace(1, 2, 300, 32, 64, 64, 0)
+
+
 def test_backward_rejects_bad_arguments(lib):
     need = lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 64, 64, 0)
     assert need > 0 and lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 64, 0, 0) == 0
     # CUDA-core backward (float32, and bf16 with chunks the tensor cores do not
     # tile): float32 forward and gradient states plus two [c][c] score blocks
     # per chunk of c = min(chunk, 128) tokens
-    for dt, chunk, c in ((0, 64, 64), (0, 37, 37), (0, 512, 128), (1, 64, 64), (1, 37, 37)):
+    for dt, chunk, c in ((0, 64, 64), (0, 37, 37), (0, 512, 128), (1, 37, 37), (1, 100, 100)):
         nc = -(-300 // c)
         assert lib.ret_chunkwise_backward_workspace(1, 2, 300, 64, 96, chunk, dt) == \
             2 * 4 * 2 * nc * (64 * 96 + c * c)
@@ -197,7 +212,7 @@ def test_backward_rejects_bad_arguments(lib):
     # float32 states, then the workspace of the forward calls (the larger of
     # the two mapped shapes), each region rounded up to 256 bytes
     al = lambda x: -(-x // 256) * 256
-    for chunk in (128, 512):
+    for chunk in (64, 128, 512):
         fws = max(lib.ret_chunkwise_workspace(1, 2, 300, 96, 64, chunk, 1),
                   lib.ret_chunkwise_workspace(1, 2, 300, 64, 96, chunk, 1))
         want = (2 * al(2 * 300 * 64 * 2) + 2 * al(2 * 300 * 96 * 2) + 4 * al(2 * 64 * 96 * 4)

@@ -100,6 +100,8 @@ CHUNK_CASES = [
     ("bf16", 2, 2, 640, 128, 128, 256, 1e-5, False),
     ("bf16", 1, 2, 1100, 128, 512, 256, None, True),
     ("bf16", 2, 3, 600, 64, 256, 128, None, True),     # d_k 64: state boxes past d_k skipped
+    ("bf16", 1, 3, 300, 256, 512, 64, 1e-5, True),     # chunk 64: tensor cores, 128-token tiles
+    ("bf16", 2, 2, 333, 128, 128, 64, None, False),
     ("bf16", 10, 4, 600, 256, 512, 256, 1e-5, False),  # 160 column tiles: both d_k halves per CTA
     ("f32", 1, 3, 301, 128, 64, 37, None, True),
     ("f32", 2, 2, 200, 64, 96, 64, 1e-5, False),
@@ -140,13 +142,13 @@ def test_chunkwise_parity_without_final_state(torch_cuda, ret, case):
     assert _rel(o, o_ref) <= TOL[dt]
 
 
-# bf16 shapes outside the tensor-core tiling (chunk not in {128, 256, 512}, or
+# bf16 shapes outside the tensor-core tiling (chunk not in {64, 128, 256, 512}, or
 # d_k / d_v not a power of two in [64, 256] / [64, 512]) run the float32
 # CUDA-core kernels on the bf16 inputs; their only rounding is the bf16
 # output, so they are held to a tolerance well inside the bf16 one.
 OFF_TC_CASES = [
     # B, H, N, dk, dv, chunk, gn_eps, state_in
-    (1, 3, 300, 256, 512, 64, 1e-5, True),    # chunk 64
+    (1, 3, 300, 256, 512, 32, 1e-5, True),    # chunk 32
     (2, 2, 333, 128, 128, 100, None, False),  # chunk not a power of two
     (1, 2, 200, 32, 64, 128, None, True),     # d_k below the tensor-core tiles
     (1, 2, 150, 512, 128, 128, None, False),  # d_k above them
@@ -470,6 +472,7 @@ BWD_CASES = [
     ("f32", 1, 3, 257, 128, 128, 128, True, False),
     ("bf16", 1, 2, 700, 128, 256, 256, True, True),
     ("bf16", 1, 2, 333, 256, 512, 512, False, False),
+    ("bf16", 1, 2, 300, 128, 256, 64, True, True),     # chunk 64: forward calls on 128-token tiles
 ]
 
 
