@@ -124,6 +124,41 @@ def test_chunkwise_parity(torch_cuda, ret, case):
     assert _rel(s, s_ref) <= STATE_TOL
 
 
+def _random_chunk_cases(n, seed):
+    """Seeded random tensor-core shapes: ragged lengths, every supported
+    d_k, d_v and chunk, GroupNorm, incoming and returned states mixed."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for _ in range(n):
+        dk = int(rng.choice([64, 128, 256]))
+        dv = int(rng.choice([64, 128, 256, 512]))
+        chunk = int(rng.choice([64, 128, 256, 512]))
+        N = int(rng.integers(1, 1600))
+        B, H = int(rng.integers(1, 3)), int(rng.integers(1, 4))
+        gn = 1e-5 if rng.random() < 0.5 else None
+        out.append((B, H, N, dk, dv, chunk, gn, bool(rng.random() < 0.5), bool(rng.random() < 0.5)))
+    return out
+
+
+@pytest.mark.parametrize("case", _random_chunk_cases(16, 2024), ids=lambda c: "-".join(map(str, c)))
+def test_chunkwise_random_tensor_core_shapes(torch_cuda, ret, case):
+    torch = torch_cuda
+    B, H, N, dk, dv, chunk, gn, with_s0, want_s = case
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=300 + N, with_state=with_s0)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    g = _gam(torch, inp["gammas"])
+    s0 = _dev(inp["state"]) if with_s0 else None
+    if want_s:
+        o, s = ret.chunkwise(q, k, v, g, chunk, state_in=s0, return_state=True, gn_eps=gn)
+    else:
+        o, s = ret.chunkwise(q, k, v, g, chunk, state_in=s0, gn_eps=gn), None
+    torch.cuda.synchronize()
+    o_ref, s_ref = _ref_chunkwise(inp, chunk, gn, with_s0)
+    assert _rel(o, o_ref) <= TOL["bf16"]
+    if want_s:
+        assert _rel(s, s_ref) <= STATE_TOL
+
+
 @pytest.mark.parametrize("case", [c for c in CHUNK_CASES if c[0] == "bf16"],
                          ids=lambda c: "-".join(map(str, c)))
 def test_chunkwise_parity_without_final_state(torch_cuda, ret, case):
@@ -603,6 +638,27 @@ def test_parallel_parity(torch_cuda, ret, case):
     if gn is not None:
         o_ref = oracle.group_norm(o_ref, gn)
     assert _rel(o, o_ref) <= TOL[dt]
+
+
+def _random_parallel_cases(n, seed):
+    rng = np.random.default_rng(seed)
+    return [(int(rng.integers(1, 3)), int(rng.integers(1, 4)), int(rng.integers(1, 1300)),
+             int(rng.choice([64, 128, 256])), int(rng.choice([64, 128, 256, 512])),
+             1e-5 if rng.random() < 0.5 else None) for _ in range(n)]
+
+
+@pytest.mark.parametrize("case", _random_parallel_cases(8, 2025), ids=lambda c: "-".join(map(str, c)))
+def test_parallel_random_tensor_core_shapes(torch_cuda, ret, case):
+    torch = torch_cuda
+    B, H, N, dk, dv, gn = case
+    inp = wl.make_inputs(B, H, N, dk, dv, "bf16", seed=400 + N)
+    q, k, v = _dev(inp["q"]), _dev(inp["k"]), _dev(inp["v"])
+    o = ret.parallel(q, k, v, _gam(torch, inp["gammas"]), gn_eps=gn)
+    torch.cuda.synchronize()
+    o_ref, _ = oracle.parallel(inp["q"].exact, inp["k"].exact, inp["v"].exact, inp["gammas"])
+    if gn is not None:
+        o_ref = oracle.group_norm(o_ref, gn)
+    assert _rel(o, o_ref) <= TOL["bf16"]
 
 
 # --- decode step -------------------------------------------------------------------
