@@ -343,15 +343,21 @@ def run_reference(args):
         return 0
     from linear_recurrent_sequence_scale_b200 import workloads as wl
     w = wl.WORKLOADS[WORKLOAD]
-    # size each step so that warmup + steps end within about two minutes
-    _, _, t1 = oracle_sample(1, 0.0)
-    heads = max(1, min(w.B * w.H, int(120.0 / max(t1, 1e-3) / max(1, args.steps + args.warmup))))
+    # size each step so that warmup + steps end within about two minutes of
+    # wall time (drawing a head's inputs costs about what the oracle does);
+    # the timed figure counts the oracle's own time only, since the GPU arm's
+    # inputs are resident before its timed region starts
+    oracle_sample(1, 0.0)  # first call: imports and allocator warm-up
+    t_wall = time.perf_counter()
+    oracle_sample(1, 0.0)
+    per_head = time.perf_counter() - t_wall
+    heads = max(1, min(w.B * w.H,
+                       int(120.0 / max(per_head, 1e-3) / max(1, args.steps + args.warmup))))
     for _ in range(args.warmup):
         oracle_sample(heads, 1e9)
-    t0 = time.perf_counter()
+    dt = 0.0
     for _ in range(args.steps):
-        oracle_sample(heads, 1e9)
-    dt = time.perf_counter() - t0
+        dt += oracle_sample(heads, 1e9)[2]
     value = heads * w.N / w.H * args.steps / dt
     cores = blas_threads()
     sample = (f"{heads} of {w.B * w.H} (batch, head) pairs of the {WORKLOAD} workload per step, "
