@@ -357,6 +357,10 @@ int ret_chunkwise_backward(const void* q, const void* k, const void* v, const fl
     const int s2 = (call);                       \
     if (s2 != RET_OK) return s2;                 \
   } while (0)
+  // the forward calls' own checks (e.g. the chunk-count limit) before any
+  // launch, so that a failing status still means nothing ran
+  RET_TRY_STATUS(check_chunkwise(B, H, N, dv, dk, RET_BF16, chunk, gammas, fws, L.fws_bytes));
+  RET_TRY_STATUS(check_chunkwise(B, H, N, dk, dv, RET_BF16, chunk, gammas, fws, L.fws_bytes));
   RET_TRY(ret::launch_reverse_rows(q, qr, BH, N, dk, st));
   RET_TRY(ret::launch_reverse_rows(k, kr, BH, N, dk, st));
   RET_TRY(ret::launch_reverse_rows(v, vr, BH, N, dv, st));

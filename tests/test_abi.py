@@ -234,6 +234,13 @@ def test_backward_rejects_bad_arguments(lib):
     assert call(ws=None) == ret.RET_EWORKSPACE
     assert call(wsb=need - 1) == ret.RET_EWORKSPACE
     assert call(N=0, q=None, dO=None, gq=None, ds=None, ws=None, wsb=0) == ret.RET_OK
+    # bf16 on the tensor cores: a sequence past the forward kernels' chunk-count
+    # limit is refused before the row reversals launch (a failing status means
+    # nothing ran; this process has no GPU, so a launch would fail otherwise)
+    n_big = 128 * 65535 + 1
+    big = lib.ret_chunkwise_backward_workspace(1, 2, n_big, 64, 64, 128, 1)
+    assert big > 0
+    assert call(N=n_big, chunk=128, dt=1, wsb=big) == ret.RET_EUNSUPPORTED
 
 
 def test_selftest_rejects_bad_limits(lib):
